@@ -1,0 +1,423 @@
+"""Benchmark: sparse decode steps/s per layer at 128K, B=2048 (one decode step =
+group-mean scoring of the projected-key cache, top-B selection and indexed
+attention for every query head; batch 4, 32 query heads, 8 KV heads, d=128,
+T=131072, r=64).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). Timing: CUDA events on the launching stream,
+W untimed warm-up steps, then K timed steps bracketed by a barrier and
+torch.cuda.synchronize() on both sides; max over ranks. Inputs (2.5 GiB per
+GPU) exceed the 126 MB L2 and every step streams the 512 MiB projected-key
+cache, so no separate L2 flush is needed.
+
+Multi-GPU: the decode step shards by sequence and KV head with no exchange, so
+each rank runs its own full workload (weak scaling, no data-path collective);
+`value` is the steps of all ranks divided by the slowest rank's time.
+
+--impl reference times the CPU oracle (fp64 NumPy) on this host's cores on a
+bounded sample of the same workload (one (sequence, KV head) unit per step),
+scaled to whole decode steps.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse decode steps/s per layer at 128K, B=2048; achieved HBM GB/s vs peak"
+UNIT = "steps/s"
+WORKLOAD = "decode_128k"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+SCORER_SOURCES = ["indexed_sparse_attention_kv_b200/csrc/score.cu",
+                  "indexed_sparse_attention_kv_b200/csrc/lsa_common.cuh"]
+
+
+def rank_seed(w, rank):
+    """Each rank decodes its own sequences: a distinct seed per rank."""
+    return w.seed + 7919 * rank
+
+
+def max_over_ranks(values, world, device=None):
+    """Elementwise max of a list of floats over all ranks (identity at world 1)."""
+    import torch
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def weak_value(world, steps, ms):
+    """Steps of all ranks divided by the slowest rank's time (steps/s)."""
+    return world * steps / (ms / 1e3)
+
+
+def _env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def config_dict(w, extra=None):
+    d = {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "d": w.d, "T": w.T, "r": w.r,
+         "B": w.B, "heavy_hitters": w.heavy_frac, "kv_layout": "[batch, T, hkv, d] bf16",
+         "l2": "inputs exceed L2 (each step streams the 512 MiB projected-key cache)"}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def algorithmic_bytes(w):
+    """Bytes the method must move per decode step: projected-key cache, the
+    selected K and V rows, q, the projected queries and out."""
+    kt = w.batch * w.T * w.hkv * w.r * 2
+    kv = w.batch * w.hkv * w.B * w.d * 2 * 2
+    small = w.batch * w.hq * (w.d * 2 + w.r * 2 + w.d * 2)
+    return kt, kv, small
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def scorer_traffic(w):
+    """DRAM bytes per scorer launch from the committed ncu summary, or None if
+    the scorer's sources changed since it was captured."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            t = json.load(f)
+        if t.get("source_hash") != source_hash(SCORER_SOURCES) or t.get("workload") != w.name:
+            return None
+        return float(t["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def blas_threads():
+    try:
+        import numpy as np
+        import threadpoolctl
+        np.ones((64, 64)) @ np.ones((64, 64))
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=1)
+        return int(n)
+    except Exception:
+        return 1
+
+
+def cpu_oracle_sample(w, x, budget_s=12.0, max_units=None):
+    """Time the oracle on (sequence, KV head) units of the workload until about
+    budget_s seconds of CPU work; returns (steps/s, units, seconds)."""
+    import numpy as np
+    import torch
+
+    import oracle.lsa_oracle as O
+
+    units_per_step = w.batch * w.hkv
+    done, t0 = 0, time.perf_counter()
+    elapsed = 0.0
+    G = w.G
+    while True:
+        b = (done // w.hkv) % w.batch
+        h = done % w.hkv
+        # one unit: the oracle's steps for one KV head of one sequence
+        qt = x["qt"][b, h * G:(h + 1) * G].to(torch.float32).numpy()
+        kt = x["kt"][b, :, h:h + 1].to(torch.float32).numpy()
+        q = x["q"][b, h * G:(h + 1) * G].to(torch.float32).numpy()
+        ts = time.perf_counter()
+        q_bar = O.group_mean_query(qt, 1)
+        s = O.candidate_scores(q_bar, kt)
+        idx = O.select_top_b(s[0], w.B)[None]
+        sel = idx[0][idx[0] >= 0]
+        k_rows = x["k"][b, sel, h:h + 1].to(torch.float32).numpy()
+        v_rows = x["v"][b, sel, h:h + 1].to(torch.float32).numpy()
+        O.indexed_attention(q, k_rows, v_rows, np.arange(len(sel))[None], w.scale)
+        elapsed += time.perf_counter() - ts
+        done += 1
+        if elapsed >= budget_s or (max_units and done >= max_units):
+            break
+        if time.perf_counter() - t0 > 3 * budget_s:
+            break
+    return done / units_per_step / elapsed, done, elapsed
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the CPU oracle as it stands, on this host's cores."""
+    if rank != 0:
+        return 0
+    from indexed_sparse_attention_kv_b200 import inputs as I
+
+    w = I.workload(WORKLOAD)
+    x = I.make_decode_inputs(w)
+    cores = blas_threads()
+    # warm-up: W units; timed: K steps, each one (sequence, KV head) unit
+    cpu_oracle_sample(w, x, budget_s=0.0, max_units=max(1, args.warmup))
+    per_unit = []
+    for _ in range(args.steps):
+        v, n, el = cpu_oracle_sample(w, x, budget_s=0.0, max_units=1)
+        per_unit.append(el)
+    unit_s = sum(per_unit) / len(per_unit)
+    step_s = unit_s * w.batch * w.hkv
+    value = 1.0 / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} timed (sequence, KV head) units of 32 per step, scaled x32"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import indexed_sparse_attention_kv_b200 as lsa
+    from indexed_sparse_attention_kv_b200 import _lib
+    from indexed_sparse_attention_kv_b200 import inputs as I
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    lsa.lib()
+    w = I.workload(WORKLOAD)
+    x = I.make_decode_inputs(w, seed=rank_seed(w, rank))
+    d = {k: x[k].to(dev) for k in ("q", "qt", "k", "v", "kt")}
+    dims = _lib.decode_dims(d["q"], d["qt"], d["k"])
+    ws = lsa.workspace(dims, w.B, device=dev)
+    idx = torch.empty((w.batch, w.hkv, w.B), dtype=torch.int32, device=dev)
+    out = torch.empty_like(d["q"])
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lsa.lsa_decode_step(d["q"], d["qt"], d["k"], d["v"], d["kt"], w.B, idx_out=idx, out=out, ws=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    status = lsa.lsa_read_device_status(ws)
+
+    # ---- timed region: K whole decode steps
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = e0.elapsed_time(e1)
+    clocks = clk.summary()
+
+    # ---- component split (Fig. 9-style): scoring / top-B / attention, events between calls
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    comp = [0.0, 0.0, 0.0]
+    scores = torch.empty((w.batch, w.hkv, w.T), dtype=torch.float32, device=dev)
+    n_comp = max(3, min(args.steps, 20))
+    for it in range(n_comp + 2):
+        ev[0].record(stream)
+        lsa.lsa_score(d["qt"], d["kt"], scores)
+        ev[1].record(stream)
+        lsa.lsa_topk(scores, w.B, idx)
+        ev[2].record(stream)
+        lsa.lsa_indexed_attn(d["q"], d["k"], d["v"], idx, out=out, ws=ws)
+        ev[3].record(stream)
+        torch.cuda.synchronize()
+        if it >= 2:
+            for j in range(3):
+                comp[j] += ev[j].elapsed_time(ev[j + 1])
+    comp = [c / n_comp for c in comp]
+
+    # ---- end to end through the public API: H2D q, qt from pinned host, step, D2H out and idx
+    hq = x["q"].pin_memory()
+    hqt = x["qt"].pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hidx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    for _ in range(2):
+        d["q"].copy_(hq, non_blocking=True)
+        d["qt"].copy_(hqt, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+        hidx.copy_(idx, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        d["q"].copy_(hq, non_blocking=True)
+        d["qt"].copy_(hqt, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+        hidx.copy_(idx, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = e0.elapsed_time(e1)
+
+    # ---- max over ranks
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
+
+    if rank == 0:
+        value = weak_value(world, args.steps, ms)
+        e2e = weak_value(world, args.steps, ms_e2e)
+        kt_b, kv_b, small_b = algorithmic_bytes(w)
+        peak, peak_kind = measured_peak()
+        score_ms = comp[0]
+        scorer_bytes = kt_b + w.batch * w.hq * w.r * 2
+        achieved = scorer_bytes / (score_ms / 1e3) / 1e9
+        traffic = scorer_traffic(w)
+        step_bytes = kt_b + kv_b + small_b
+        step_gbs = step_bytes / (ms / args.steps / 1e3) / 1e9
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            v, n, el = cpu_oracle_sample(w, x, budget_s=args.cpu_budget)
+            cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                   "sample": f"{n} (sequence, KV head) units of the 128K workload ({el:.1f} s), scaled to steps"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_dict(w, {"parallelism": f"replicas{world}" if world > 1 else "single"}),
+            "roofline": {"bound": "hbm", "kernel": "score_flat_kernel", "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": scorer_bytes,
+                         "avg_launch_ms": score_ms},
+            "step_roofline": {"achieved": step_gbs, "peak": peak, "unit": "GB/s", "frac": step_gbs / peak,
+                              "algorithmic_bytes_per_step": step_bytes},
+            "components_ms": {"scoring": comp[0], "top_b": comp[1], "attention": comp[2]},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e, "unit": UNIT,
+                    "h2d_bytes_per_step": hq.numel() * 2 + hqt.numel() * 2,
+                    "d2h_bytes_per_step": hout.numel() * 2 + hidx.numel() * 4},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    rank = _env_int("RANK", 0)
+    world = _env_int("WORLD_SIZE", 1)
+    local_rank = _env_int("LOCAL_RANK", 0)
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

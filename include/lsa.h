@@ -1,0 +1,196 @@
+/*
+ * lsa.h — C ABI of liblsa.so: indexed sparse attention over a GQA KV cache on
+ * NVIDIA B200 (sm_100a).
+ *
+ * One decode step, per sequence b and KV head h (Joint Subspace Sparse
+ * Attention for Efficient Long-Context Decoding, Fig. 1 and Key contributions):
+ *   q_bar[b,h]  = mean of the projected queries qt[b,i] of h's query group
+ *   s[b,h,t]    = q_bar[b,h] . kt[b,t,h]            for every cached t
+ *   S[b,h]      = top-B positions of s[b,h,:]       (ties: lower position)
+ *   out[b,i]    = softmax attention of q[b,i] over K/V rows S[b,h], read in
+ *                 place from the [T, hkv, d] cache (no gather copy)
+ * optionally coarse-to-fine over block centroids first (LongCat Sparse
+ * Attention: Taming the Lightning via Streaming-aware Hierarchical Cross-Layer
+ * Indexing, Abstract, strategy (3) Hierarchical Indexing), plus the prefill
+ * indexer (the same scoring and top-B for every query row of a prefill, causal)
+ * and prefill indexed attention.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers, owned by the caller. The library
+ *     never allocates, frees or synchronizes; every call enqueues its kernels on
+ *     `stream` (a cudaStream_t passed as void*, NULL = legacy default stream)
+ *     and returns at once.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     validation failure returns a negative lsa_status and launches nothing.
+ *   - Pointers must be 16-byte aligned and tensors densely packed, row-major,
+ *     in the layouts given below. bf16 tensors are passed as lsa_bf16 (raw
+ *     16-bit storage of bfloat16 values).
+ *   - GQA grouping: query head i belongs to KV head i / G, G = hq / hkv.
+ *   - Index sets are int32, strictly ascending, padded at the end with -1 when
+ *     fewer than B candidates exist. NaN scores mark non-candidates.
+ *   - Supported sizes: r in {16, 32, 64, 128}; d in {64, 128, 256};
+ *     1 <= hkv, hkv * r <= 4096; G = hq / hkv in {1, 2, 4, 8, 16};
+ *     1 <= T <= 2^31 - 1; 1 <= B <= 65536. Other sizes return
+ *     LSA_ERR_UNSUPPORTED.
+ *   - Errors found on the device (an index outside [-1, T), a bounded wait that
+ *     ran out) are OR-ed into a status word at the start of the workspace;
+ *     read it with lsa_read_device_status. Kernels never trap.
+ */
+#ifndef LSA_H
+#define LSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LSA_API __attribute__((visibility("default")))
+#else
+#define LSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int lsa_status;
+enum {
+    LSA_OK = 0,
+    LSA_ERR_ARG = -1,         /* null pointer, non-positive size, hq % hkv != 0 */
+    LSA_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned */
+    LSA_ERR_SHAPE = -3,       /* inconsistent sizes (e.g. q_start + nq > T) */
+    LSA_ERR_WORKSPACE = -4,   /* workspace missing, misaligned (256 B) or too small */
+    LSA_ERR_CUDA = -5,        /* a CUDA launch failed (cudaGetLastError) */
+    LSA_ERR_TIMEOUT = -6,     /* reserved: device-side bounded wait ran out (status word) */
+    LSA_ERR_UNSUPPORTED = -7  /* sizes outside the supported set above */
+};
+
+/* Bits of the device status word (lsa_read_device_status). */
+enum {
+    LSA_DEV_OK = 0,
+    LSA_DEV_BAD_INDEX = 1,    /* an index outside [-1, T) was skipped */
+    LSA_DEV_TIMEOUT = 2       /* a bounded wait ran out; outputs are incomplete */
+};
+
+typedef uint16_t lsa_bf16;
+
+/* Problem sizes. batch sequences, hq query heads, hkv KV heads, head dim d,
+ * scoring-subspace rank r (the projected-key cache width), cache length T. */
+typedef struct lsa_dims {
+    int batch, hq, hkv, d, r, T;
+} lsa_dims;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+LSA_API int lsa_version(void);
+
+/* Human-readable name of a status code. Never NULL. */
+LSA_API const char* lsa_status_string(lsa_status s);
+
+/* Bytes of workspace needed by lsa_topk, lsa_indexed_attn and lsa_decode_step
+ * for these sizes. blk = tokens per block and nblk_keep = blocks kept in
+ * coarse-to-fine mode; pass 0, 0 for flat scoring. Returns 0 for invalid
+ * sizes. The workspace must be 256-byte aligned; its contents need no
+ * initialisation except the status word (lsa_clear_device_status). */
+LSA_API size_t lsa_workspace_size(const lsa_dims* dims, int B, int blk, int nblk_keep);
+
+/* Group-mean candidate scoring (JSSA, Fig. 1; Fig. 2a "channel budget r").
+ *   qt     [batch, hq, r]      bf16  projected queries
+ *   kt     [batch, T, hkv, r]  bf16  projected-key cache
+ *   scores [batch, hkv, T]     fp32  out: q_bar[b,h] . kt[b,t,h]
+ * q_bar is the mean of the group's projected queries; the group sum is formed
+ * in fp32, the dot product accumulates in fp32, and the result is divided by G
+ * (exact when G is a power of two). Integer-valued inputs give exact scores. */
+LSA_API lsa_status lsa_score(const lsa_dims* dims, const lsa_bf16* qt, const lsa_bf16* kt,
+                     float* scores, void* stream);
+
+/* Top-B selection per row (JSSA, Fig. 1 "select the top-B token positions").
+ *   scores [batch * hkv, T] fp32   one row per (b, h); NaN = not a candidate
+ *   idx    [batch * hkv, B] int32  out: the B positions with the largest
+ *          scores, ties broken toward the lower position, ascending, -1 padded
+ * ws may be NULL (ws_bytes 0); if given, its status word is not touched.
+ * -0.0 and +0.0 compare equal. Deterministic: identical inputs give identical
+ * outputs. */
+LSA_API lsa_status lsa_topk(const lsa_dims* dims, const float* scores, int B, int32_t* idx,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* Gather-free indexed attention (JSSA, Key contributions; Fig. 1).
+ *   q    [batch, hq, d]      bf16
+ *   k, v [batch, T, hkv, d]  bf16  the standard GQA KV cache, read in place
+ *   idx  [batch, hkv, B]     int32 per-KV-head index sets (-1 entries skipped)
+ *   out  [batch, hq, d]      bf16  out: softmax(scale * q . K[S]) V[S], fp32
+ *                                  accumulation, rounded to nearest even
+ * Entries outside [-1, T) are skipped and set LSA_DEV_BAD_INDEX. A head whose
+ * set is empty gets a zero output. ws: lsa_workspace_size(dims, B, 0, 0). */
+LSA_API lsa_status lsa_indexed_attn(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* k,
+                            const lsa_bf16* v, const int32_t* idx, int B, float scale,
+                            lsa_bf16* out, void* ws, size_t ws_bytes, void* stream);
+
+/* One whole decode step: scoring, top-B and indexed attention (JSSA, Fig. 1).
+ *   q [batch, hq, d], qt [batch, hq, r], k/v [batch, T, hkv, d],
+ *   kt [batch, T, hkv, r]: as above.
+ *   centroids  NULL for flat scoring; else [batch, ceil(T/blk), hkv, r] bf16
+ *              block centroids (lsa_block_centroids) for coarse-to-fine mode:
+ *              score the centroids, keep the nblk_keep best blocks (ties: the
+ *              lower block), score the tokens of those blocks, take the top B
+ *              (LongCat Sparse Attention, Abstract, strategy (3)).
+ *   idx_out    NULL, or [batch, hkv, B] int32 to receive the index sets.
+ *   out        [batch, hq, d] bf16.
+ * Selection inside the step ranks the group-sum scores (G times the mean),
+ * which orders positions exactly as the mean does. */
+LSA_API lsa_status lsa_decode_step(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* qt,
+                           const lsa_bf16* k, const lsa_bf16* v, const lsa_bf16* kt,
+                           const lsa_bf16* centroids, int blk, int nblk_keep, int B,
+                           float scale, int32_t* idx_out, lsa_bf16* out,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Block centroids for coarse-to-fine scoring (LongCat Sparse Attention,
+ * Abstract, strategy (3); Latent Sparse Attention, summary: queries score
+ * clusters instead of every key).
+ *   kt        [batch, T, hkv, r]           bf16
+ *   centroids [batch, ceil(T/blk), hkv, r] bf16  out: sum of the block's
+ *             (up to blk) projected keys, fp32 sum rounded to nearest even
+ * blk in [1, 4096]. Blocks start at t = 0; the last one may be partial. */
+LSA_API lsa_status lsa_block_centroids(const lsa_dims* dims, const lsa_bf16* kt, int blk,
+                               lsa_bf16* centroids, void* stream);
+
+/* Bytes of workspace for lsa_prefill_index / lsa_prefill_attn. */
+LSA_API size_t lsa_prefill_workspace_size(const lsa_dims* dims, int nq, int B);
+
+/* Prefill indexer (LongCat Sparse Attention, Abstract: the Lightning Indexer's
+ * dense O(L^2) scoring; JSSA, Fig. 1 for the group-mean query): for each of nq
+ * query rows at absolute positions q_start .. q_start + nq - 1, score every
+ * key t <= p with the row's group mean and take the top B (causal).
+ *   dims.batch must be 1; dims.T = cache length (the queries' own keys are in
+ *   the cache, so q_start + nq <= T).
+ *   qt  [nq, hq, r]   bf16     kt [T, hkv, r] bf16
+ *   idx [nq, hkv, B]  int32    out, ascending, -1 padded (rows with p+1 < B)
+ * The group mean is rounded to bf16 for the tensor-core contraction (exact when
+ * it is a multiple of 2^-k representable in bf16, e.g. integer inputs). */
+LSA_API lsa_status lsa_prefill_index(const lsa_dims* dims, const lsa_bf16* qt, int nq, int q_start,
+                             const lsa_bf16* kt, int B, int32_t* idx,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Prefill indexed attention: lsa_indexed_attn for each of nq query rows, the
+ * G heads of a KV head sharing that row's index set.
+ *   q [nq, hq, d], k/v [T, hkv, d], idx [nq, hkv, B], out [nq, hq, d]. */
+LSA_API lsa_status lsa_prefill_attn(const lsa_dims* dims, const lsa_bf16* q, int nq,
+                            const lsa_bf16* k, const lsa_bf16* v, const int32_t* idx, int B,
+                            float scale, lsa_bf16* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Enqueue a copy of the workspace's device status word into *host_flags
+ * (pinned or pageable host memory); synchronize `stream` before reading it. */
+LSA_API lsa_status lsa_read_device_status(const void* ws, int32_t* host_flags, void* stream);
+
+/* Enqueue a reset of the workspace's device status word to LSA_DEV_OK. */
+LSA_API lsa_status lsa_clear_device_status(void* ws, void* stream);
+
+/* Test hook: the number of failed polls after which a device-side wait gives
+ * up and sets LSA_DEV_TIMEOUT (default 1 << 26; negative restores it). It
+ * affects only launches enqueued after the call. Process-wide, not
+ * thread-safe. */
+LSA_API void lsa_debug_set_wait_limit(long long polls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H */

@@ -1,0 +1,24 @@
+"""Indexed sparse attention over a GQA KV cache for NVIDIA B200 (sm_100a).
+
+The compute lives in liblsa.so (hand-written CUDA, C ABI in include/lsa.h);
+this package is its Python binding (``_lib``) and the seeded synthetic inputs
+(``inputs``). Importing the package does not load the library; the first call
+does, and raises if liblsa.so has not been built.
+"""
+from ._lib import (  # noqa: F401
+    LsaError,
+    lib,
+    lsa_block_centroids,
+    lsa_clear_device_status,
+    lsa_debug_set_wait_limit,
+    lsa_decode_step,
+    lsa_dims,
+    lsa_indexed_attn,
+    lsa_read_device_status,
+    lsa_score,
+    lsa_topk,
+    lsa_workspace_size,
+    workspace,
+)
+
+__version__ = "0.1.0"

@@ -1,0 +1,283 @@
+// C-ABI layer of liblsa.so: argument validation, workspace layout and launch
+// sequencing on the caller's stream. Declarations and contracts: include/lsa.h.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/lsa.h"
+#include "lsa_internal.h"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kHeaderBytes = 256;       // device status word + reserved
+constexpr long long kDefaultWaitLimit = 1ll << 26;
+
+std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
+
+int device_sms() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+lsa::LaunchCtx make_ctx(void* stream) {
+    lsa::LaunchCtx c;
+    c.stream = reinterpret_cast<cudaStream_t>(stream);
+    c.num_sms = device_sms();
+    c.wait_limit = g_wait_limit.load();
+    return c;
+}
+
+lsa_status check_dims(const lsa_dims* d) {
+    if (!d) return LSA_ERR_ARG;
+    if (d->batch < 1 || d->hq < 1 || d->hkv < 1 || d->d < 1 || d->r < 1 || d->T < 1) return LSA_ERR_ARG;
+    if (d->hq % d->hkv != 0) return LSA_ERR_ARG;
+    const int G = d->hq / d->hkv;
+    if (!pow2_in(G, 1, 16)) return LSA_ERR_UNSUPPORTED;
+    if (!(d->r == 16 || d->r == 32 || d->r == 64 || d->r == 128)) return LSA_ERR_UNSUPPORTED;
+    if (!(d->d == 64 || d->d == 128 || d->d == 256)) return LSA_ERR_UNSUPPORTED;
+    if ((long long)d->hkv * d->r > 4096) return LSA_ERR_UNSUPPORTED;
+    return LSA_OK;
+}
+
+lsa_status check_B(int B) {
+    if (B < 1) return LSA_ERR_ARG;
+    if (B > 65536) return LSA_ERR_UNSUPPORTED;
+    return LSA_OK;
+}
+
+lsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA; }
+
+// Workspace layout (byte offsets from the 256-byte aligned base).
+struct DecodeLayout {
+    size_t status = 0;        // uint32 device status word
+    size_t scores = 0;        // fp32 [batch, hkv, T]   (flat) or coarse [batch, hkv, nblk]
+    size_t fine = 0;          // fp32 [batch, hkv, keep * blk]  (hierarchical)
+    size_t blkidx = 0;        // int32 [batch, hkv, keep]       (hierarchical)
+    size_t idx = 0;           // int32 [batch, hkv, B]
+    size_t pm = 0, pl = 0, po = 0;
+    size_t total = 0;
+    lsa::AttnPlan plan{};
+};
+
+DecodeLayout decode_layout(const lsa_dims* d, int B, int blk, int keep, int num_sms) {
+    DecodeLayout L;
+    size_t off = kHeaderBytes;
+    const size_t units = (size_t)d->batch * d->hkv;
+    const size_t nscore = blk > 0 ? (size_t)(d->T + blk - 1) / blk : (size_t)d->T;
+    L.scores = off;
+    off = align_up(off + units * nscore * 4);
+    if (blk > 0) {
+        L.fine = off;
+        off = align_up(off + units * (size_t)keep * blk * 4);
+        L.blkidx = off;
+        off = align_up(off + units * (size_t)keep * 4);
+    }
+    L.idx = off;
+    off = align_up(off + units * (size_t)B * 4);
+    const int G = d->hq / d->hkv;
+    L.plan = lsa::plan_attn(d->batch, d->hkv, G, B, num_sms);
+    const size_t heads = (size_t)d->batch * d->hq;
+    L.pm = off;
+    off = align_up(off + heads * L.plan.nsw * 4);
+    L.pl = off;
+    off = align_up(off + heads * L.plan.nsw * 4);
+    L.po = off;
+    off = align_up(off + heads * L.plan.nsw * (size_t)d->d * 4);
+    L.total = off;
+    return L;
+}
+
+lsa_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
+    if (!ws) return LSA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return LSA_ERR_WORKSPACE;
+    if (ws_bytes < need) return LSA_ERR_WORKSPACE;
+    return LSA_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+}  // namespace
+
+extern "C" {
+
+int lsa_version(void) { return 100; }
+
+const char* lsa_status_string(lsa_status s) {
+    switch (s) {
+        case LSA_OK: return "LSA_OK";
+        case LSA_ERR_ARG: return "LSA_ERR_ARG: invalid argument (null pointer or bad size)";
+        case LSA_ERR_ALIGN: return "LSA_ERR_ALIGN: pointer not 16-byte aligned";
+        case LSA_ERR_SHAPE: return "LSA_ERR_SHAPE: inconsistent sizes";
+        case LSA_ERR_WORKSPACE: return "LSA_ERR_WORKSPACE: workspace missing, misaligned or too small";
+        case LSA_ERR_CUDA: return "LSA_ERR_CUDA: a CUDA launch failed";
+        case LSA_ERR_TIMEOUT: return "LSA_ERR_TIMEOUT: a device-side wait ran out";
+        case LSA_ERR_UNSUPPORTED: return "LSA_ERR_UNSUPPORTED: sizes outside the supported set";
+        default: return "LSA_ERR_UNKNOWN";
+    }
+}
+
+void lsa_debug_set_wait_limit(long long polls) { g_wait_limit.store(polls < 0 ? kDefaultWaitLimit : polls); }
+
+size_t lsa_workspace_size(const lsa_dims* dims, int B, int blk, int nblk_keep) {
+    if (check_dims(dims) != LSA_OK || check_B(B) != LSA_OK) return 0;
+    if (blk < 0 || nblk_keep < 0 || (blk > 0) != (nblk_keep > 0)) return 0;
+    return decode_layout(dims, B, blk, nblk_keep, device_sms()).total;
+}
+
+lsa_status lsa_score(const lsa_dims* dims, const lsa_bf16* qt, const lsa_bf16* kt, float* scores, void* stream) {
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if (!qt || !kt || !scores) return LSA_ERR_ARG;
+    if (!aligned16(qt) || !aligned16(kt) || !aligned16(scores)) return LSA_ERR_ALIGN;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    return from_cuda(lsa::launch_score(ctx, qt, kt, scores, dims->batch, dims->hq, dims->hkv, dims->r, dims->T, 1,
+                                       nullptr));
+}
+
+lsa_status lsa_topk(const lsa_dims* dims, const float* scores, int B, int32_t* idx, void* ws, size_t ws_bytes,
+                    void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if ((s = check_B(B)) != LSA_OK) return s;
+    if (!scores || !idx) return LSA_ERR_ARG;
+    if (!aligned16(scores) || !aligned16(idx)) return LSA_ERR_ALIGN;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    return from_cuda(
+        lsa::launch_topk(ctx, scores, dims->batch * dims->hkv, dims->T, B, idx, nullptr, 0, 0));
+}
+
+lsa_status lsa_indexed_attn(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* k, const lsa_bf16* v,
+                            const int32_t* idx, int B, float scale, lsa_bf16* out, void* ws, size_t ws_bytes,
+                            void* stream) {
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if ((s = check_B(B)) != LSA_OK) return s;
+    if (!q || !k || !v || !idx || !out) return LSA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(out)) return LSA_ERR_ALIGN;
+    if (!std::isfinite(scale)) return LSA_ERR_ARG;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    const DecodeLayout L = decode_layout(dims, B, 0, 0, ctx.num_sms);
+    if ((s = check_ws(ws, ws_bytes, L.total)) != LSA_OK) return s;
+    return from_cuda(lsa::launch_attn(ctx, L.plan, q, k, v, idx, B, scale, out, at<float>(ws, L.pm),
+                                      at<float>(ws, L.pl), at<float>(ws, L.po), dims->batch, dims->hq, dims->hkv,
+                                      dims->d, dims->T, (long long)dims->T * dims->hkv,
+                                      at<unsigned>(ws, L.status)));
+}
+
+lsa_status lsa_decode_step(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* qt, const lsa_bf16* k,
+                           const lsa_bf16* v, const lsa_bf16* kt, const lsa_bf16* centroids, int blk, int nblk_keep,
+                           int B, float scale, int32_t* idx_out, lsa_bf16* out, void* ws, size_t ws_bytes,
+                           void* stream) {
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if ((s = check_B(B)) != LSA_OK) return s;
+    if (!q || !qt || !k || !v || !kt || !out) return LSA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(qt) || !aligned16(k) || !aligned16(v) || !aligned16(kt) || !aligned16(out))
+        return LSA_ERR_ALIGN;
+    if (idx_out && !aligned16(idx_out)) return LSA_ERR_ALIGN;
+    if (!std::isfinite(scale)) return LSA_ERR_ARG;
+    const bool hier = centroids != nullptr;
+    if (hier) {
+        if (!aligned16(centroids)) return LSA_ERR_ALIGN;
+        if (blk < 1 || blk > 4096 || nblk_keep < 1) return LSA_ERR_ARG;
+        if ((long long)nblk_keep * blk > (1ll << 24)) return LSA_ERR_UNSUPPORTED;
+        const int nblk = (dims->T + blk - 1) / blk;
+        if (nblk_keep > nblk) nblk_keep = nblk;
+    } else {
+        blk = 0;
+        nblk_keep = 0;
+    }
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    const DecodeLayout L = decode_layout(dims, B, blk, nblk_keep, ctx.num_sms);
+    if ((s = check_ws(ws, ws_bytes, L.total)) != LSA_OK) return s;
+    unsigned* status = at<unsigned>(ws, L.status);
+    int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
+    const int rows = dims->batch * dims->hkv;
+    cudaError_t e;
+    if (!hier) {
+        e = lsa::launch_score(ctx, qt, kt, at<float>(ws, L.scores), dims->batch, dims->hq, dims->hkv, dims->r, dims->T,
+                              0, status);
+        if (e == cudaSuccess) e = lsa::launch_topk(ctx, at<float>(ws, L.scores), rows, dims->T, B, idx, nullptr, 0, 0);
+    } else {
+        const int nblk = (dims->T + blk - 1) / blk;
+        int32_t* blkidx = at<int32_t>(ws, L.blkidx);
+        float* fine = at<float>(ws, L.fine);
+        e = lsa::launch_score(ctx, qt, centroids, at<float>(ws, L.scores), dims->batch, dims->hq, dims->hkv, dims->r,
+                              nblk, 0, status);
+        if (e == cudaSuccess)
+            e = lsa::launch_topk(ctx, at<float>(ws, L.scores), rows, nblk, nblk_keep, blkidx, nullptr, 0, 0);
+        if (e == cudaSuccess)
+            e = lsa::launch_fine_score(ctx, qt, kt, blkidx, nblk_keep, blk, fine, dims->batch, dims->hq, dims->hkv,
+                                       dims->r, dims->T);
+        if (e == cudaSuccess)
+            e = lsa::launch_topk(ctx, fine, rows, nblk_keep * blk, B, idx, blkidx, blk, nblk_keep);
+    }
+    if (e == cudaSuccess)
+        e = lsa::launch_attn(ctx, L.plan, q, k, v, idx, B, scale, out, at<float>(ws, L.pm), at<float>(ws, L.pl),
+                             at<float>(ws, L.po), dims->batch, dims->hq, dims->hkv, dims->d, dims->T,
+                             (long long)dims->T * dims->hkv, status);
+    return from_cuda(e);
+}
+
+lsa_status lsa_block_centroids(const lsa_dims* dims, const lsa_bf16* kt, int blk, lsa_bf16* centroids, void* stream) {
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if (!kt || !centroids) return LSA_ERR_ARG;
+    if (blk < 1 || blk > 4096) return LSA_ERR_ARG;
+    if (!aligned16(kt) || !aligned16(centroids)) return LSA_ERR_ALIGN;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    return from_cuda(lsa::launch_centroids(ctx, kt, blk, centroids, dims->batch, dims->hkv, dims->r, dims->T));
+}
+
+size_t lsa_prefill_workspace_size(const lsa_dims* dims, int nq, int B) {
+    (void)dims;
+    (void)nq;
+    (void)B;
+    return 0;
+}
+
+lsa_status lsa_prefill_index(const lsa_dims* dims, const lsa_bf16* qt, int nq, int q_start, const lsa_bf16* kt, int B,
+                             int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+    (void)dims; (void)qt; (void)nq; (void)q_start; (void)kt; (void)B; (void)idx; (void)ws; (void)ws_bytes;
+    (void)stream;
+    return LSA_ERR_UNSUPPORTED;
+}
+
+lsa_status lsa_prefill_attn(const lsa_dims* dims, const lsa_bf16* q, int nq, const lsa_bf16* k, const lsa_bf16* v,
+                            const int32_t* idx, int B, float scale, lsa_bf16* out, void* ws, size_t ws_bytes,
+                            void* stream) {
+    (void)dims; (void)q; (void)nq; (void)k; (void)v; (void)idx; (void)B; (void)scale; (void)out; (void)ws;
+    (void)ws_bytes; (void)stream;
+    return LSA_ERR_UNSUPPORTED;
+}
+
+lsa_status lsa_read_device_status(const void* ws, int32_t* host_flags, void* stream) {
+    if (!ws || !host_flags) return LSA_ERR_ARG;
+    return from_cuda(cudaMemcpyAsync(host_flags, ws, sizeof(int32_t), cudaMemcpyDeviceToHost,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lsa_status lsa_clear_device_status(void* ws, void* stream) {
+    if (!ws) return LSA_ERR_ARG;
+    return from_cuda(cudaMemsetAsync(ws, 0, sizeof(int32_t), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,42 @@
+// Internal launchers shared by the kernel files and the C-ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace lsa {
+
+struct LaunchCtx {
+    cudaStream_t stream;
+    int num_sms;
+    long long wait_limit;
+};
+
+struct AttnPlan {
+    int rpc;      // index-set entries per CTA
+    int splits;   // CTAs per (row, KV head)
+    int nsw;      // partial slots per query head
+};
+
+// mode 0: scores are the group-sum dot products (G x the mean); mode 1: means.
+cudaError_t launch_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_t* kt, float* out, int batch, int hq,
+                         int hkv, int r, int n, int mode, unsigned* status);
+
+cudaError_t launch_fine_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_t* kt, const int32_t* blk_idx,
+                              int keep, int blk, float* out, int batch, int hq, int hkv, int r, int T);
+
+cudaError_t launch_centroids(const LaunchCtx& ctx, const uint16_t* kt, int blk, uint16_t* cen, int batch, int hkv, int r,
+                             int T);
+
+cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int n, int B, int32_t* idx,
+                        const int32_t* blkmap, int blk, int keep);
+
+AttnPlan plan_attn(int nb, int hkv, int G, int B, int num_sms);
+
+cudaError_t launch_attn(const LaunchCtx& ctx, const AttnPlan& plan, const uint16_t* q, const uint16_t* k,
+                        const uint16_t* v, const int32_t* idx, int B, float scale, uint16_t* out, float* pm, float* pl,
+                        float* po, int nb, int hq, int hkv, int d, int T, long long kv_bstride_rows,
+                        unsigned* status);
+
+}  // namespace lsa

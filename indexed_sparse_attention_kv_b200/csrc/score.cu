@@ -1,0 +1,349 @@
+// Candidate scoring kernels: flat streaming scorer, fine (candidate-list)
+// scorer for coarse-to-fine mode, and block centroids.
+//
+// Joint Subspace Sparse Attention for Efficient Long-Context Decoding, Fig. 1:
+// for each KV head, the mean of its query group scores every row of a
+// projected-key cache [T, hkv, r]. The scorer is an HBM stream: every byte of
+// the projected-key cache is read once, through 1-D TMA bulk copies into a
+// multi-stage shared-memory ring, and reduced with fp32 FMAs.
+#include <cuda_bf16.h>
+
+#include "lsa_common.cuh"
+#include "lsa_internal.h"
+
+namespace lsa {
+
+namespace {
+
+constexpr int kScoreThreads = 256;
+constexpr int kScoreWarps = kScoreThreads / 32;
+constexpr int kScoreStages = 4;
+constexpr int kChunkTarget = 16384;   // bytes per pipeline stage (approximate)
+constexpr long long kDrainPolls = 1ll << 26;
+
+struct ScoreArgs {
+    const uint16_t* qt;    // [batch, hq, r]
+    const uint8_t* kt;     // [batch, n, hkv, r] bf16
+    float* out;            // [batch, hkv, n]
+    int hq, hkv, n, G;
+    int tok_per_chunk;     // tokens per stage, multiple of the tokens per warp pass
+    int chunks_per_batch;
+    int ctas_per_batch;
+    int mode;              // 0: group sum, 1: group mean
+    int g_pow2;
+    float inv_g;
+    unsigned* status;
+    long long wait_limit;
+};
+
+__device__ __forceinline__ float finalize_score(float acc, const ScoreArgs& a) {
+    if (a.mode == 0) return acc;
+    return a.g_pow2 ? acc * a.inv_g : __fdiv_rn(acc, (float)a.G);
+}
+
+__device__ __forceinline__ float dot8(const uint4 w, const float* q) {
+    float acc = 0.f;
+    acc = fmaf(q[0], bf16lo(w.x), acc);
+    acc = fmaf(q[1], bf16hi(w.x), acc);
+    acc = fmaf(q[2], bf16lo(w.y), acc);
+    acc = fmaf(q[3], bf16hi(w.y), acc);
+    acc = fmaf(q[4], bf16lo(w.z), acc);
+    acc = fmaf(q[5], bf16hi(w.z), acc);
+    acc = fmaf(q[6], bf16lo(w.w), acc);
+    acc = fmaf(q[7], bf16hi(w.w), acc);
+    return acc;
+}
+
+// One CTA streams a contiguous range of chunks of one sequence. A chunk is
+// tok_per_chunk whole tokens (all hkv heads, r channels each). A warp pass
+// covers TPW consecutive tokens of one head: LPR = r/8 lanes per row, each lane
+// 16 bytes, so a pass reads TPW rows and writes TPW consecutive scores.
+template <int R, bool FIXED_HEAD>
+__global__ void __launch_bounds__(kScoreThreads) score_flat_kernel(const ScoreArgs a) {
+    constexpr int LPR = R / 8;
+    constexpr int TPW = 32 / LPR;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int hkv = a.hkv;
+    const int row_bytes = R * 2;
+    const int token_bytes = hkv * row_bytes;
+    const int chunk_bytes = a.tok_per_chunk * token_bytes;
+    uint8_t* stages = smem;
+    float* qbar = reinterpret_cast<float*>(smem + kScoreStages * chunk_bytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(qbar + hkv * R);
+
+    const int b = blockIdx.y;
+    const int c0 = (int)((long long)blockIdx.x * a.chunks_per_batch / a.ctas_per_batch);
+    const int c1 = (int)((long long)(blockIdx.x + 1) * a.chunks_per_batch / a.ctas_per_batch);
+    const int nch = c1 - c0;
+    const uint8_t* kt_b = a.kt + (size_t)b * a.n * token_bytes;
+
+    // Group-sum query of every KV head (fp32; exact for integer-valued bf16).
+    for (int e = threadIdx.x; e < hkv * R; e += kScoreThreads) {
+        const int h = e / R, j = e - h * R;
+        const uint16_t* src = a.qt + ((size_t)b * a.hq + (size_t)h * a.G) * R + j;
+        float s = 0.f;
+        for (int g = 0; g < a.G; ++g) s += __uint_as_float(((uint32_t)src[(size_t)g * R]) << 16);
+        qbar[e] = s;
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kScoreStages; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    auto issue = [&](int i) {
+        const int t0 = (c0 + i) * a.tok_per_chunk;
+        const int ntok = min(a.tok_per_chunk, a.n - t0);
+        const uint32_t bytes = (uint32_t)(ntok * token_bytes);
+        uint64_t* bar = &bars[i % kScoreStages];
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(stages + (i % kScoreStages) * chunk_bytes, kt_b + (size_t)t0 * token_bytes, bytes, bar);
+    };
+    if (threadIdx.x == 0) {
+        const int npro = min(kScoreStages, nch);
+        for (int i = 0; i < npro; ++i) issue(i);
+    }
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / LPR;      // token within the warp pass
+    const int cpart = lane % LPR;    // 16-byte column chunk of the row
+    float qreg[8];
+    if (FIXED_HEAD) {
+        const float* qs = qbar + (warp % hkv) * R + cpart * 8;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) qreg[k] = qs[k];
+    }
+    const int items = hkv * (a.tok_per_chunk / TPW);
+    float* out_b = a.out + (size_t)b * hkv * a.n;
+
+    int i = 0;
+    bool timed_out = false;
+    for (; i < nch; ++i) {
+        const int s = i % kScoreStages;
+        const bool ready = mbar_wait_bounded(&bars[s], (uint32_t)((i / kScoreStages) & 1), a.wait_limit);
+        if (!__syncthreads_and(ready)) {
+            timed_out = true;
+            break;
+        }
+        const int t0 = (c0 + i) * a.tok_per_chunk;
+        const int ntok = min(a.tok_per_chunk, a.n - t0);
+        const uint8_t* st = stages + s * chunk_bytes;
+        for (int item = warp; item < items; item += kScoreWarps) {
+            const int h = FIXED_HEAD ? (warp % hkv) : (item % hkv);
+            const int tl = (item / hkv) * TPW + sub;
+            float acc = 0.f;
+            if (tl < ntok) {
+                const uint4 w = *reinterpret_cast<const uint4*>(st + (size_t)tl * token_bytes + h * row_bytes + cpart * 16);
+                if (FIXED_HEAD) {
+                    acc = dot8(w, qreg);
+                } else {
+                    float qv[8];
+                    const float* qs = qbar + h * R + cpart * 8;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) qv[k] = qs[k];
+                    acc = dot8(w, qv);
+                }
+            }
+#pragma unroll
+            for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (cpart == 0 && tl < ntok) out_b[(size_t)h * a.n + t0 + tl] = finalize_score(acc, a);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0 && i + kScoreStages < nch) issue(i + kScoreStages);
+    }
+    if (timed_out) {
+        // Leave no bulk copy in flight into this CTA's shared memory.
+        if (threadIdx.x == 0) {
+            set_status(a.status, kStatusTimeout);
+            const int issued = min(nch, i + kScoreStages);
+            for (int j = i; j < issued; ++j)
+                mbar_wait_bounded(&bars[j % kScoreStages], (uint32_t)((j / kScoreStages) & 1), kDrainPolls);
+        }
+        __syncthreads();
+    }
+}
+
+// Fine scorer for coarse-to-fine mode: candidate c of (b, h) is token
+// blk_idx[b,h,c / blk] * blk + c % blk; scores go to out[b, h, c], NaN for a
+// padded block or a token past T. Direct 16-byte loads (rows are scattered).
+struct FineArgs {
+    const uint16_t* qt;
+    const uint8_t* kt;
+    const int32_t* blk_idx;   // [batch, hkv, keep]
+    float* out;               // [batch, hkv, keep * blk]
+    int hq, hkv, T, G, blk, keep, ncand;
+};
+
+template <int R>
+__global__ void __launch_bounds__(256) score_fine_kernel(const FineArgs a) {
+    constexpr int LPR = R / 8;
+    constexpr int TPW = 32 / LPR;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / LPR, cpart = lane % LPR;
+    float q[8];
+    {
+        const uint16_t* src = a.qt + ((size_t)b * a.hq + (size_t)h * a.G) * R + cpart * 8;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) q[k] = 0.f;
+        for (int g = 0; g < a.G; ++g)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) q[k] += __uint_as_float(((uint32_t)src[(size_t)g * R + k]) << 16);
+    }
+    const int32_t* bi = a.blk_idx + ((size_t)b * a.hkv + h) * a.keep;
+    float* out = a.out + ((size_t)b * a.hkv + h) * a.ncand;
+    const size_t row_stride = (size_t)a.hkv * R * 2;
+    const uint8_t* base = a.kt + (size_t)b * a.T * row_stride + (size_t)h * R * 2 + cpart * 16;
+    const int per_cta = (a.ncand + gridDim.x - 1) / gridDim.x;
+    const int cbeg = blockIdx.x * per_cta, cend = min(a.ncand, cbeg + per_cta);
+    for (int c_base = cbeg + warp * TPW; c_base < cend; c_base += 8 * TPW) {
+        const int c = c_base + sub;
+        bool valid = false;
+        float acc = 0.f;
+        if (c < cend) {
+            const int j = c / a.blk;
+            const int blkid = bi[j];
+            const long long pos = (long long)blkid * a.blk + (c - j * a.blk);
+            valid = blkid >= 0 && pos < a.T;
+            if (valid) acc = dot8(ldg_stream16(base + (size_t)pos * row_stride), q);
+        }
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (cpart == 0 && c < cend) out[c] = valid ? acc : __int_as_float(0x7fc00000);
+    }
+}
+
+// Block centroids: c[b, j, h, :] = sum over the block's tokens of kt[b, t, h, :].
+// One CTA per (block, sequence); thread i owns 8 consecutive channels of the
+// [hkv * r] token row.
+__global__ void __launch_bounds__(512) centroid_kernel(const uint8_t* kt, uint16_t* cen, int T, int blk, int row_elems,
+                                                        int nblk) {
+    const int j = blockIdx.x, b = blockIdx.y;
+    const int i = threadIdx.x;
+    if (i * 8 >= row_elems) return;
+    const size_t row_bytes = (size_t)row_elems * 2;
+    const uint8_t* src = kt + ((size_t)b * T + (size_t)j * blk) * row_bytes + (size_t)i * 16;
+    const int ntok = min(blk, T - j * blk);
+    float acc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+    for (int t = 0; t < ntok; ++t) {
+        const uint4 w = ldg_stream16(src + (size_t)t * row_bytes);
+        acc[0] += bf16lo(w.x); acc[1] += bf16hi(w.x);
+        acc[2] += bf16lo(w.y); acc[3] += bf16hi(w.y);
+        acc[4] += bf16lo(w.z); acc[5] += bf16hi(w.z);
+        acc[6] += bf16lo(w.w); acc[7] += bf16hi(w.w);
+    }
+    uint4 o;
+    o.x = (uint32_t)f2bf(acc[0]) | ((uint32_t)f2bf(acc[1]) << 16);
+    o.y = (uint32_t)f2bf(acc[2]) | ((uint32_t)f2bf(acc[3]) << 16);
+    o.z = (uint32_t)f2bf(acc[4]) | ((uint32_t)f2bf(acc[5]) << 16);
+    o.w = (uint32_t)f2bf(acc[6]) | ((uint32_t)f2bf(acc[7]) << 16);
+    *reinterpret_cast<uint4*>(cen + ((size_t)b * nblk + j) * row_elems + (size_t)i * 8) = o;
+}
+
+template <int R, bool FIXED>
+cudaError_t launch_flat_t(const LaunchCtx& ctx, ScoreArgs a, int batch) {
+    constexpr int LPR = R / 8;
+    constexpr int TPW = 32 / LPR;
+    const int token_bytes = a.hkv * R * 2;
+    int tok = kChunkTarget / token_bytes;
+    tok = tok < TPW ? TPW : (tok / TPW) * TPW;
+    a.tok_per_chunk = tok;
+    a.chunks_per_batch = (a.n + tok - 1) / tok;
+    const size_t smem = (size_t)kScoreStages * tok * token_bytes + (size_t)a.hkv * R * 4 + kScoreStages * 8;
+    auto kern = score_flat_kernel<R, FIXED>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kScoreThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) occ = 1;
+    const long long target = (long long)ctx.num_sms * occ;
+    long long per_b = (target + batch - 1) / batch;
+    if (per_b > a.chunks_per_batch) per_b = a.chunks_per_batch;
+    if (per_b < 1) per_b = 1;
+    a.ctas_per_batch = (int)per_b;
+    dim3 grid((unsigned)per_b, (unsigned)batch);
+    kern<<<grid, kScoreThreads, smem, ctx.stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <int R>
+cudaError_t launch_flat_r(const LaunchCtx& ctx, const ScoreArgs& a, int batch) {
+    const bool fixed = (kScoreWarps % a.hkv) == 0;
+    return fixed ? launch_flat_t<R, true>(ctx, a, batch) : launch_flat_t<R, false>(ctx, a, batch);
+}
+
+template <int R>
+cudaError_t launch_fine_r(const LaunchCtx& ctx, const FineArgs& a, int batch) {
+    constexpr int TPW = 32 / (R / 8);
+    const int per_cta_target = 8 * TPW * 8;   // eight warp passes per warp
+    int ctas = (a.ncand + per_cta_target - 1) / per_cta_target;
+    if (ctas < 1) ctas = 1;
+    dim3 grid((unsigned)ctas, (unsigned)a.hkv, (unsigned)batch);
+    score_fine_kernel<R><<<grid, 256, 0, ctx.stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_t* kt, float* out, int batch, int hq,
+                         int hkv, int r, int n, int mode, unsigned* status) {
+    ScoreArgs a{};
+    a.qt = qt;
+    a.kt = reinterpret_cast<const uint8_t*>(kt);
+    a.out = out;
+    a.hq = hq;
+    a.hkv = hkv;
+    a.n = n;
+    a.G = hq / hkv;
+    a.mode = mode;
+    a.g_pow2 = (a.G & (a.G - 1)) == 0;
+    a.inv_g = 1.0f / (float)a.G;
+    a.status = status;
+    a.wait_limit = ctx.wait_limit;
+    switch (r) {
+        case 16: return launch_flat_r<16>(ctx, a, batch);
+        case 32: return launch_flat_r<32>(ctx, a, batch);
+        case 64: return launch_flat_r<64>(ctx, a, batch);
+        case 128: return launch_flat_r<128>(ctx, a, batch);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_fine_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_t* kt, const int32_t* blk_idx,
+                              int keep, int blk, float* out, int batch, int hq, int hkv, int r, int T) {
+    FineArgs a{};
+    a.qt = qt;
+    a.kt = reinterpret_cast<const uint8_t*>(kt);
+    a.blk_idx = blk_idx;
+    a.out = out;
+    a.hq = hq;
+    a.hkv = hkv;
+    a.T = T;
+    a.G = hq / hkv;
+    a.blk = blk;
+    a.keep = keep;
+    a.ncand = keep * blk;
+    switch (r) {
+        case 16: return launch_fine_r<16>(ctx, a, batch);
+        case 32: return launch_fine_r<32>(ctx, a, batch);
+        case 64: return launch_fine_r<64>(ctx, a, batch);
+        case 128: return launch_fine_r<128>(ctx, a, batch);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_centroids(const LaunchCtx& ctx, const uint16_t* kt, int blk, uint16_t* cen, int batch, int hkv, int r,
+                             int T) {
+    const int row_elems = hkv * r;
+    const int nblk = (T + blk - 1) / blk;
+    int threads = ((row_elems / 8) + 31) / 32 * 32;
+    dim3 grid((unsigned)nblk, (unsigned)batch);
+    centroid_kernel<<<grid, threads, 0, ctx.stream>>>(reinterpret_cast<const uint8_t*>(kt), cen, T, blk, row_elems,
+                                                      nblk);
+    return cudaGetLastError();
+}
+
+}  // namespace lsa

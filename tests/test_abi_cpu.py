@@ -1,0 +1,95 @@
+"""Host-only checks of liblsa.so: it loads, exports every function lsa.h
+declares, and rejects bad arguments before launching anything (no GPU needed:
+every call below fails validation on the host)."""
+import ctypes
+
+import pytest
+
+import indexed_sparse_attention_kv_b200._lib as L
+
+pytestmark = pytest.mark.skipif(not __import__("os").path.exists(L.LIB_PATH), reason="liblsa.so not built")
+
+ALIGNED = ctypes.c_void_p(1 << 20)      # never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p((1 << 20) + 8)
+
+
+def test_exports_every_declared_symbol():
+    names = L.header_functions()
+    assert len(names) >= 14
+    lib = L.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(L._SIGS), set(names) ^ set(L._SIGS)
+
+
+def test_version_and_status_strings():
+    lib = L.lib()
+    assert lib.lsa_version() == 100
+    for code, name in L.STATUS_NAMES.items():
+        assert lib.lsa_status_string(code).decode().startswith(name)
+    assert lib.lsa_status_string(-99).decode() == "LSA_ERR_UNKNOWN"
+
+
+def _dims(**kw):
+    base = dict(batch=1, hq=4, hkv=1, d=128, r=64, T=4096)
+    base.update(kw)
+    return L.make_dims(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(batch=0), -1), (dict(hq=0), -1), (dict(T=0), -1), (dict(hq=6, hkv=4), -1),
+    (dict(hq=12, hkv=4), -7), (dict(r=48), -7), (dict(d=96), -7), (dict(hq=64, hkv=64, r=128), -7),
+])
+def test_bad_dims(kw, code):
+    lib = L.lib()
+    d = _dims(**kw)
+    assert lib.lsa_score(ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, None) == code
+    assert lib.lsa_workspace_size(ctypes.byref(d), 256, 0, 0) == 0
+
+
+def test_null_and_alignment():
+    lib = L.lib()
+    d = _dims()
+    assert lib.lsa_score(None, ALIGNED, ALIGNED, ALIGNED, None) == -1
+    assert lib.lsa_score(ctypes.byref(d), None, ALIGNED, ALIGNED, None) == -1
+    assert lib.lsa_score(ctypes.byref(d), MISALIGNED, ALIGNED, ALIGNED, None) == -2
+    assert lib.lsa_topk(ctypes.byref(d), ALIGNED, 0, ALIGNED, None, 0, None) == -1
+    assert lib.lsa_topk(ctypes.byref(d), ALIGNED, 70000, ALIGNED, None, 0, None) == -7
+    assert lib.lsa_topk(ctypes.byref(d), MISALIGNED, 16, ALIGNED, None, 0, None) == -2
+    f = ctypes.c_float
+    assert lib.lsa_indexed_attn(ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, None, 16, f(0.1), ALIGNED,
+                                ALIGNED, 1 << 30, None) == -1
+    assert lib.lsa_indexed_attn(ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, ALIGNED, 16, f(float("nan")),
+                                ALIGNED, ALIGNED, 1 << 30, None) == -1
+    assert lib.lsa_block_centroids(ctypes.byref(d), ALIGNED, 0, ALIGNED, None) == -1
+    assert lib.lsa_block_centroids(ctypes.byref(d), ALIGNED, 64, MISALIGNED, None) == -2
+    assert lib.lsa_read_device_status(None, ALIGNED, None) == -1
+    assert lib.lsa_clear_device_status(None, None) == -1
+
+
+def test_workspace_checks():
+    lib = L.lib()
+    d = _dims()
+    need = lib.lsa_workspace_size(ctypes.byref(d), 256, 0, 0)
+    assert need > 0 and need % 256 == 0
+    # coarse-to-fine: block scores + candidate scores + block ids replace the T scores
+    hier = lib.lsa_workspace_size(ctypes.byref(d), 256, 64, 16)
+    assert hier > 0 and hier % 256 == 0 and hier != need
+    assert lib.lsa_workspace_size(ctypes.byref(d), 256, 64, 0) == 0
+    f = ctypes.c_float
+    args = (ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, ALIGNED, 256, f(0.1), ALIGNED)
+    assert lib.lsa_indexed_attn(*args, None, need, None) == -4
+    assert lib.lsa_indexed_attn(*args, ctypes.c_void_p((1 << 20) + 16), need, None) == -4
+    assert lib.lsa_indexed_attn(*args, ALIGNED, need - 1, None) == -4
+    step = lib.lsa_decode_step
+    assert step(ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 0, 0, 256, f(0.1), None,
+                ALIGNED, ALIGNED, 16, None) == -4
+    assert step(ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 0, 16, 256, f(0.1), None,
+                ALIGNED, ALIGNED, 1 << 30, None) == -1     # centroids given, blk = 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        L.lsa_score(q[:, :, :64], torch.zeros(1, 8, 1, 64, dtype=torch.bfloat16))
