@@ -387,6 +387,38 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def run_ncu_case(args):
+    """A small, self-contained launch sequence for ncu captures: batch 2 of the
+    128K workload (kt 256 MiB > L2, 1.3 GiB on the device), `--steps` launches
+    of the chosen component after `--warmup` untimed ones."""
+    import torch
+
+    import indexed_sparse_attention_kv_b200 as lsa
+    from indexed_sparse_attention_kv_b200 import _lib
+    from indexed_sparse_attention_kv_b200 import inputs as I
+
+    w = I.workload(WORKLOAD).with_(batch=2, name="decode_128k_b2")
+    x = I.make_decode_inputs(w)
+    d = {k: x[k].cuda() for k in ("q", "qt", "k", "v", "kt")}
+    dims = _lib.decode_dims(d["q"], d["qt"], d["k"])
+    ws = lsa.workspace(dims, w.B)
+    scores = lsa.lsa_score(d["qt"], d["kt"])
+    idx = lsa.lsa_topk(scores, w.B)
+    out = torch.empty_like(d["q"])
+    fn = {
+        "score": lambda: lsa.lsa_score(d["qt"], d["kt"], scores),
+        "topk": lambda: lsa.lsa_topk(scores, w.B, idx),
+        "attn": lambda: lsa.lsa_indexed_attn(d["q"], d["k"], d["v"], idx, out=out, ws=ws),
+        "step": lambda: lsa.lsa_decode_step(d["q"], d["qt"], d["k"], d["v"], d["kt"], w.B, idx_out=idx, out=out,
+                                            ws=ws),
+    }[args.ncu_case]
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize()
+    print(f"ncu case {args.ncu_case}: {args.warmup}+{args.steps} launches, status {lsa.lsa_read_device_status(ws)}")
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -395,7 +427,11 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu-case", choices=["score", "topk", "attn", "step"], default=None,
+                    help="run one component on a reduced 128K case (batch 2) for an ncu capture; no JSON")
     args = ap.parse_args(argv)
+    if args.ncu_case:
+        return run_ncu_case(args)
     rank = _env_int("RANK", 0)
     world = _env_int("WORLD_SIZE", 1)
     local_rank = _env_int("LOCAL_RANK", 0)
