@@ -40,6 +40,7 @@ METRIC = "sparse decode steps/s per layer at 128K, B=2048; achieved HBM GB/s vs 
 UNIT = "steps/s"
 WORKLOAD = "decode_128k"
 FALLBACK_HBM_GBS = 6650.0
+KERNELS_PER_STEP = 3      # scorer, top-B, indexed attention (split combine fused into it)
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 SCORER_SOURCES = ["indexed_sparse_attention_kv_b200/csrc/score.cu",
                   "indexed_sparse_attention_kv_b200/csrc/lsa_common.cuh"]
@@ -123,54 +124,73 @@ def scorer_traffic(w):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """SM clock, power and clock-event (throttle) reasons sampled through NVML
+    (the library nvidia-smi reads) every ~2 ms in a thread while the timed
+    region runs; read-only."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    def __init__(self, torch_device):
+        self.dev = torch_device
+        self.rows = []
+        self.err = None
+        self._stop = None
+        self._thr = None
+
+    def _handle(self, nv):
+        import torch
+
+        try:
+            p = torch.cuda.get_device_properties(self.dev)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
 
     def __enter__(self):
+        import threading
+
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml as nv
+
+            nv.nvmlInit()
+            h = self._handle(nv)
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report it, do not guess
+            self.err = f"nvml unavailable: {type(e).__name__}"
+            return self
+        self._stop = threading.Event()
+
+        def loop():
+            while True:
+                try:
+                    self.rows.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), int(get_reasons(h)),
+                                      nv.nvmlDeviceGetPowerUsage(h) / 1e3))
+                except Exception as e:
+                    self.err = f"nvml sample failed: {type(e).__name__}"
+                    return
+                if self._stop.wait(0.002):
+                    return
+
+        self._thr = threading.Thread(target=loop, daemon=True)
+        self._thr.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        if self._thr is not None:
+            self._stop.set()
+            self._thr.join(timeout=5)
 
     def summary(self):
-        if self.proc is None or not self.path:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "no samples"], "samples": 0}
+        reasons = sorted({name for _, r, _ in self.rows for bit, name in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(m for m, _, _ in self.rows), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.rows),
+                "power_w_max": max(p for _, _, p in self.rows), "source": "nvml"}
 
 
 def blas_threads():
@@ -284,39 +304,68 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     status = lsa.lsa_read_device_status(ws)
 
+    def graph_of(fn, reps=1):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        return g
+
+    # one decode step (3 kernel launches) captured once, replayed K times
+    g_step = graph_of(step)
+    for _ in range(max(3, args.warmup)):
+        g_step.replay()
+    torch.cuda.synchronize()
+
     # ---- timed region: K whole decode steps
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(dev) as clk:
         barrier()
         torch.cuda.synchronize()
         e0.record(stream)
         for _ in range(args.steps):
-            step()
+            g_step.replay()
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
     ms = e0.elapsed_time(e1)
     clocks = clk.summary()
 
-    # ---- component split (Fig. 9-style): scoring / top-B / attention, events between calls
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-    comp = [0.0, 0.0, 0.0]
+    # ---- component split (Fig. 9-style): each public call replayed back to back
+    # in its own graph; attention is timed after an L2 flush (as in a real step,
+    # where the scorer's 512 MiB stream has evicted the K/V rows), the flush
+    # alone timed the same way and subtracted.
     scores = torch.empty((w.batch, w.hkv, w.T), dtype=torch.float32, device=dev)
-    n_comp = max(3, min(args.steps, 20))
-    for it in range(n_comp + 2):
-        ev[0].record(stream)
-        lsa.lsa_score(d["qt"], d["kt"], scores)
-        ev[1].record(stream)
-        lsa.lsa_topk(scores, w.B, idx)
-        ev[2].record(stream)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    lsa.lsa_score(d["qt"], d["kt"], scores)
+    lsa.lsa_topk(scores, w.B, idx)
+    lsa.lsa_indexed_attn(d["q"], d["k"], d["v"], idx, out=out, ws=ws)
+    reps = 8
+
+    def attn_after_flush():
+        flush.zero_()
         lsa.lsa_indexed_attn(d["q"], d["k"], d["v"], idx, out=out, ws=ws)
-        ev[3].record(stream)
+
+    graphs = {
+        "scoring": graph_of(lambda: lsa.lsa_score(d["qt"], d["kt"], scores), reps),
+        "top_b": graph_of(lambda: lsa.lsa_topk(scores, w.B, idx), reps),
+        "attention+flush": graph_of(attn_after_flush, reps),
+        "flush": graph_of(lambda: flush.zero_(), reps),
+    }
+    comp_ms = {}
+    n_rep = 5
+    for name, g in graphs.items():
+        e0.record(stream)
+        for _ in range(n_rep):
+            g.replay()
+        e1.record(stream)
         torch.cuda.synchronize()
-        if it >= 2:
-            for j in range(3):
-                comp[j] += ev[j].elapsed_time(ev[j + 1])
-    comp = [c / n_comp for c in comp]
+        comp_ms[name] = e0.elapsed_time(e1) / (n_rep * reps)
+    comp = [comp_ms["scoring"], comp_ms["top_b"], max(0.0, comp_ms["attention+flush"] - comp_ms["flush"])]
+    del graphs, flush
 
     # ---- end to end through the public API: H2D q, qt from pinned host, step, D2H out and idx
     hq = x["q"].pin_memory()
@@ -379,7 +428,7 @@ def run_ours(args, rank, world, local_rank):
             "e2e": {"value": e2e, "unit": UNIT,
                     "h2d_bytes_per_step": hq.numel() * 2 + hqt.numel() * 2,
                     "d2h_bytes_per_step": hout.numel() * 2 + hidx.numel() * 4},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
             "clocks": clocks,
             "device_status": status,
         }
@@ -422,7 +471,7 @@ def run_ncu_case(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=12.0)

@@ -88,8 +88,10 @@ LSA_API const char* lsa_status_string(lsa_status s);
 /* Bytes of workspace needed by lsa_topk, lsa_indexed_attn and lsa_decode_step
  * for these sizes. blk = tokens per block and nblk_keep = blocks kept in
  * coarse-to-fine mode; pass 0, 0 for flat scoring. Returns 0 for invalid
- * sizes. The workspace must be 256-byte aligned; its contents need no
- * initialisation except the status word (lsa_clear_device_status). */
+ * sizes. The workspace must be 256-byte aligned and zero-filled before its
+ * first use (e.g. cudaMemsetAsync); every completed call leaves its internal
+ * counters at zero again, so it is reusable without re-zeroing. Calls that
+ * share one workspace must not overlap on the GPU (one stream, or ordered). */
 LSA_API size_t lsa_workspace_size(const lsa_dims* dims, int B, int blk, int nblk_keep);
 
 /* Group-mean candidate scoring (JSSA, Fig. 1; Fig. 2a "channel budget r").
@@ -183,10 +185,10 @@ LSA_API lsa_status lsa_read_device_status(const void* ws, int32_t* host_flags, v
 /* Enqueue a reset of the workspace's device status word to LSA_DEV_OK. */
 LSA_API lsa_status lsa_clear_device_status(void* ws, void* stream);
 
-/* Test hook: the number of failed polls after which a device-side wait gives
- * up and sets LSA_DEV_TIMEOUT (default 1 << 26; negative restores it). It
- * affects only launches enqueued after the call. Process-wide, not
- * thread-safe. */
+/* Test hook: nanoseconds of device time after which a device-side wait gives
+ * up and sets LSA_DEV_TIMEOUT (default 2e9; 0 = give up at the first failed
+ * probe; negative restores the default). It affects only launches enqueued
+ * after the call. Process-wide. */
 LSA_API void lsa_debug_set_wait_limit(long long polls);
 
 #ifdef __cplusplus

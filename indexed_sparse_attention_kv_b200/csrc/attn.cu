@@ -41,6 +41,8 @@ struct AttnArgs {
     int nsw;                  // partial slots per head = splits * warps per head
     float qscale;             // scale * log2(e)
     unsigned* status;
+    unsigned long long* counters;   // [nb, hkv] finished-split counters (zero between launches)
+    int splits;
 };
 
 // Swizzled position of 16-byte chunk c of tile row j: XOR bits 1..2 of the chunk
@@ -58,8 +60,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
     constexpr int RPW = kNT / WPH;             // tile rows per warp (softmax/PV)
 
     extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t* kv_s = smem;                                          // [2][2][kNT][D] bf16
-    float* qs = reinterpret_cast<float*>(smem + 2 * 2 * kNT * D * 2);   // [G][D]
+    const int nstages = a.rpc > kNT ? 2 : 1;
+    uint8_t* kv_s = smem;                                          // [nstages][2][kNT][D] bf16
+    float* qs = reinterpret_cast<float*>(smem + nstages * 2 * kNT * D * 2);   // [G][D]
     float* ps = qs + G * D;                                        // [G][kNT]
     int* rows_s = reinterpret_cast<int*>(ps + G * kNT);            // [rpc]
 
@@ -248,51 +251,62 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
             for (int k = 0; k < DPL; ++k) po[k] = o_st[hh][k];
         }
     }
+    if (a.nsw == 1) return;
+
+    // The last CTA of this (row, KV head) to finish merges every slot of its
+    // G query heads (threadfence-reduction pattern; the counter is left at 0).
+    __threadfence();
+    __syncthreads();
+    __shared__ int is_last;
+    if (tid == 0) {
+        unsigned long long* cnt = a.counters + (size_t)b * a.hkv + h;
+        const unsigned long long old = atomicAdd(cnt, 1ull);
+        is_last = old + 1 == (unsigned long long)a.splits;
+        if (is_last) atomicExch(cnt, 0ull);
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    for (int g = warp; g < G; g += kAttnWarps) {
+        const size_t w = (size_t)b * a.hq + h * G + g;
+        const float* m = a.pm + w * a.nsw;
+        const float* l = a.pl + w * a.nsw;
+        float M = -INFINITY;
+        for (int s = lane; s < a.nsw; s += 32) M = fmaxf(M, __ldcg(m + s));
+        M = warp_max(M);
+        float acc[DPL];
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
+        float L = 0.f;
+        if (M != -INFINITY) {
+            for (int s = 0; s < a.nsw; ++s) {
+                const float ms = __ldcg(m + s);
+                if (ms == -INFINITY) continue;
+                const float wgt = exp2f(ms - M);
+                L = fmaf(wgt, __ldcg(l + s), L);
+                const float* o = a.po + (w * a.nsw + s) * D + lane * DPL;
+#pragma unroll
+                for (int k = 0; k < DPL; ++k) acc[k] = fmaf(wgt, __ldcg(o + k), acc[k]);
+            }
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        uint16_t* o = a.out + w * D + lane * DPL;
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) o[k] = f2bf(acc[k] * inv);
+    }
 }
 
-// Merge the partial slots of every (row, query head): one warp each.
-template <int D>
-__global__ void __launch_bounds__(128) combine_kernel(const float* pm, const float* pl, const float* po, uint16_t* out,
-                                                      int nheads, int nsw) {
-    constexpr int DPL = D / 32;
-    const int w = blockIdx.x * 4 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (w >= nheads) return;
-    const float* m = pm + (size_t)w * nsw;
-    const float* l = pl + (size_t)w * nsw;
-    float M = -INFINITY;
-    for (int s = lane; s < nsw; s += 32) M = fmaxf(M, m[s]);
-    M = warp_max(M);
-    float acc[DPL];
-#pragma unroll
-    for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
-    float L = 0.f;
-    if (M != -INFINITY) {
-        for (int s = 0; s < nsw; ++s) {
-            const float ms = m[s];
-            if (ms == -INFINITY) continue;
-            const float wgt = exp2f(ms - M);
-            L = fmaf(wgt, l[s], L);
-            const float* o = po + ((size_t)w * nsw + s) * D + lane * DPL;
-#pragma unroll
-            for (int k = 0; k < DPL; ++k) acc[k] = fmaf(wgt, o[k], acc[k]);
-        }
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    uint16_t* o = out + (size_t)w * D + lane * DPL;
-#pragma unroll
-    for (int k = 0; k < DPL; ++k) o[k] = f2bf(acc[k] * inv);
-}
+int attn_stages(int rpc) { return rpc > kNT ? 2 : 1; }
 
 size_t attn_smem_bytes(int D, int G, int rpc) {
-    return (size_t)2 * 2 * kNT * D * 2 + (size_t)G * D * 4 + (size_t)G * kNT * 4 + (size_t)rpc * 4;
+    return (size_t)attn_stages(rpc) * 2 * kNT * D * 2 + (size_t)G * D * 4 + (size_t)G * kNT * 4 + (size_t)rpc * 4;
 }
 
 template <int D, int G>
 cudaError_t launch_attn_t(const LaunchCtx& ctx, const AttnArgs& a, int splits, int nb) {
     const size_t smem = attn_smem_bytes(D, G, a.rpc);
     auto kern = attn_kernel<D, G>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_dyn_smem((const void*)kern, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)splits, (unsigned)a.hkv, (unsigned)nb);
     kern<<<grid, kAttnThreads, smem, ctx.stream>>>(a);
@@ -314,16 +328,13 @@ cudaError_t launch_attn_d(const LaunchCtx& ctx, const AttnArgs& a, int G, int sp
 }  // namespace
 
 AttnPlan plan_attn(int nb, int hkv, int G, int B, int num_sms) {
+    // Largest slice (a multiple of one 64-row tile, at most 1024 rows) that
+    // still gives about six CTAs per SM; one-tile slices keep a single stage.
     AttnPlan p{};
     const long long units = (long long)nb * hkv;
-    const long long target = 3ll * num_sms;
-    long long splits = (target + units - 1) / units;
-    const long long max_splits = (B + kNT - 1) / kNT;
-    if (splits > max_splits) splits = max_splits;
-    if (splits < 1) splits = 1;
-    int rpc = (int)((B + splits - 1) / splits);
-    rpc = (rpc + kNT - 1) / kNT * kNT;
-    if (rpc > 1024) rpc = 1024;
+    const long long target = 6ll * num_sms;
+    int rpc = kNT;
+    while (rpc < 1024 && units * ((B + 2 * rpc - 1) / (2 * rpc)) >= target) rpc *= 2;
     p.rpc = rpc;
     p.splits = (B + rpc - 1) / rpc;
     const int wph = G >= kAttnWarps ? 1 : kAttnWarps / G;
@@ -333,8 +344,8 @@ AttnPlan plan_attn(int nb, int hkv, int G, int B, int num_sms) {
 
 cudaError_t launch_attn(const LaunchCtx& ctx, const AttnPlan& plan, const uint16_t* q, const uint16_t* k,
                         const uint16_t* v, const int32_t* idx, int B, float scale, uint16_t* out, float* pm, float* pl,
-                        float* po, int nb, int hq, int hkv, int d, int T, long long kv_bstride_rows,
-                        unsigned* status) {
+                        float* po, unsigned long long* counters, int nb, int hq, int hkv, int d, int T,
+                        long long kv_bstride_rows, unsigned* status) {
     AttnArgs a{};
     a.q = q;
     a.k = reinterpret_cast<const uint8_t*>(k);
@@ -353,23 +364,15 @@ cudaError_t launch_attn(const LaunchCtx& ctx, const AttnPlan& plan, const uint16
     a.nsw = plan.nsw;
     a.qscale = scale * kLog2e;
     a.status = status;
+    a.counters = counters;
+    a.splits = plan.splits;
     const int G = hq / hkv;
-    cudaError_t e;
     switch (d) {
-        case 64: e = launch_attn_d<64>(ctx, a, G, plan.splits, nb); break;
-        case 128: e = launch_attn_d<128>(ctx, a, G, plan.splits, nb); break;
-        case 256: e = launch_attn_d<256>(ctx, a, G, plan.splits, nb); break;
+        case 64: return launch_attn_d<64>(ctx, a, G, plan.splits, nb);
+        case 128: return launch_attn_d<128>(ctx, a, G, plan.splits, nb);
+        case 256: return launch_attn_d<256>(ctx, a, G, plan.splits, nb);
         default: return cudaErrorInvalidValue;
     }
-    if (e != cudaSuccess || plan.nsw == 1) return e;
-    const int nheads = nb * hq;
-    const unsigned blocks = (unsigned)((nheads + 3) / 4);
-    switch (d) {
-        case 64: combine_kernel<64><<<blocks, 128, 0, ctx.stream>>>(pm, pl, po, out, nheads, plan.nsw); break;
-        case 128: combine_kernel<128><<<blocks, 128, 0, ctx.stream>>>(pm, pl, po, out, nheads, plan.nsw); break;
-        case 256: combine_kernel<256><<<blocks, 128, 0, ctx.stream>>>(pm, pl, po, out, nheads, plan.nsw); break;
-    }
-    return cudaGetLastError();
 }
 
 }  // namespace lsa

@@ -14,7 +14,7 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr size_t kHeaderBytes = 256;       // device status word + reserved
-constexpr long long kDefaultWaitLimit = 1ll << 26;
+constexpr long long kDefaultWaitLimit = 2000000000ll;   // ns of device time
 
 std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
@@ -25,10 +25,13 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
 
 int device_sms() {
+    static std::atomic<int> cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev >= 0 && dev < 64 && cache[dev].load() > 0) return cache[dev].load();
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    if (dev >= 0 && dev < 64) cache[dev].store(n);
     return n;
 }
 
@@ -68,6 +71,7 @@ struct DecodeLayout {
     size_t blkidx = 0;        // int32 [batch, hkv, keep]       (hierarchical)
     size_t idx = 0;           // int32 [batch, hkv, B]
     size_t pm = 0, pl = 0, po = 0;
+    size_t counters = 0;      // uint64 [batch, hkv] attention split counters
     size_t total = 0;
     lsa::AttnPlan plan{};
 };
@@ -96,6 +100,8 @@ DecodeLayout decode_layout(const lsa_dims* d, int B, int blk, int keep, int num_
     off = align_up(off + heads * L.plan.nsw * 4);
     L.po = off;
     off = align_up(off + heads * L.plan.nsw * (size_t)d->d * 4);
+    L.counters = off;
+    off = align_up(off + units * 8);
     L.total = off;
     return L;
 }
@@ -177,7 +183,8 @@ lsa_status lsa_indexed_attn(const lsa_dims* dims, const lsa_bf16* q, const lsa_b
     const DecodeLayout L = decode_layout(dims, B, 0, 0, ctx.num_sms);
     if ((s = check_ws(ws, ws_bytes, L.total)) != LSA_OK) return s;
     return from_cuda(lsa::launch_attn(ctx, L.plan, q, k, v, idx, B, scale, out, at<float>(ws, L.pm),
-                                      at<float>(ws, L.pl), at<float>(ws, L.po), dims->batch, dims->hq, dims->hkv,
+                                      at<float>(ws, L.pl), at<float>(ws, L.po),
+                                      at<unsigned long long>(ws, L.counters), dims->batch, dims->hq, dims->hkv,
                                       dims->d, dims->T, (long long)dims->T * dims->hkv,
                                       at<unsigned>(ws, L.status)));
 }
@@ -232,7 +239,8 @@ lsa_status lsa_decode_step(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf
     }
     if (e == cudaSuccess)
         e = lsa::launch_attn(ctx, L.plan, q, k, v, idx, B, scale, out, at<float>(ws, L.pm), at<float>(ws, L.pl),
-                             at<float>(ws, L.po), dims->batch, dims->hq, dims->hkv, dims->d, dims->T,
+                             at<float>(ws, L.po), at<unsigned long long>(ws, L.counters), dims->batch, dims->hq,
+                             dims->hkv, dims->d, dims->T,
                              (long long)dims->T * dims->hkv, status);
     return from_cuda(e);
 }

@@ -64,15 +64,43 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
-// Bounded wait: polls at most `limit` times after the first failed probe
-// (backing off with nanosleep), returns false if the phase never completed.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, long long limit) {
+// Potentially blocking probe: the hardware may suspend the thread for a
+// system-dependent time before it returns false.
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait on phase `parity`: gives up after `limit_ns` nanoseconds of
+// device time (0: after the first failed probe) or as soon as *abort becomes
+// non-zero (abort may be null). Returns false if the phase did not complete.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, long long limit_ns,
+                                                  const volatile int* abort = nullptr) {
     if (mbar_test(bar, parity)) return true;
-    for (long long i = 0; i < limit; ++i) {
-        if (mbar_test(bar, parity)) return true;
-        if (i > 64) __nanosleep(64);
+    if (limit_ns <= 0) return false;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (abort && *abort) return false;
+        if ((long long)(globaltimer_ns() - t0) > limit_ns) return false;
     }
-    return false;
 }
 
 // 1-D bulk copy global -> shared through the TMA unit, completing on `bar`.

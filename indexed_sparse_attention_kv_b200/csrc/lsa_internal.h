@@ -5,7 +5,47 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <map>
+#include <mutex>
+#include <tuple>
+
 namespace lsa {
+
+// Host-side caches so that a launch costs no driver attribute queries after
+// the first call (per kernel, device and configuration).
+inline int current_device() {
+    int d = 0;
+    cudaGetDevice(&d);
+    return d;
+}
+
+inline cudaError_t ensure_dyn_smem(const void* kern, int bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, int> done;
+    const int dev = current_device();
+    std::lock_guard<std::mutex> g(mu);
+    int& cur = done[{kern, dev}];
+    if (cur >= bytes) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) cur = bytes;
+    return e;
+}
+
+inline cudaError_t cached_occupancy(const void* kern, int threads, size_t smem, int* occ) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void*, int, int, size_t>, int> done;
+    const int dev = current_device();
+    std::lock_guard<std::mutex> g(mu);
+    auto key = std::make_tuple(kern, dev, threads, smem);
+    auto it = done.find(key);
+    if (it != done.end()) {
+        *occ = it->second;
+        return cudaSuccess;
+    }
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, kern, threads, smem);
+    if (e == cudaSuccess) done[key] = *occ;
+    return e;
+}
 
 struct LaunchCtx {
     cudaStream_t stream;
@@ -34,9 +74,10 @@ cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int
 
 AttnPlan plan_attn(int nb, int hkv, int G, int B, int num_sms);
 
+// counters: [nb * hkv] zero-initialised; the kernel leaves them zero.
 cudaError_t launch_attn(const LaunchCtx& ctx, const AttnPlan& plan, const uint16_t* q, const uint16_t* k,
                         const uint16_t* v, const int32_t* idx, int B, float scale, uint16_t* out, float* pm, float* pl,
-                        float* po, int nb, int hq, int hkv, int d, int T, long long kv_bstride_rows,
-                        unsigned* status);
+                        float* po, unsigned long long* counters, int nb, int hq, int hkv, int d, int T,
+                        long long kv_bstride_rows, unsigned* status);
 
 }  // namespace lsa

@@ -19,7 +19,7 @@ constexpr int kScoreThreads = 256;
 constexpr int kScoreWarps = kScoreThreads / 32;
 constexpr int kScoreStages = 4;
 constexpr int kChunkTarget = 16384;   // bytes per pipeline stage (approximate)
-constexpr long long kDrainPolls = 1ll << 26;
+constexpr long long kDrainNs = 4000000000ll;   // 4 s: copies in flight always land
 
 struct ScoreArgs {
     const uint16_t* qt;    // [batch, hq, r]
@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_flat_kernel(const ScoreAr
             set_status(a.status, kStatusTimeout);
             const int issued = min(nch, i + kScoreStages);
             for (int j = i; j < issued; ++j)
-                mbar_wait_bounded(&bars[j % kScoreStages], (uint32_t)((j / kScoreStages) & 1), kDrainPolls);
+                mbar_wait_bounded(&bars[j % kScoreStages], (uint32_t)((j / kScoreStages) & 1), kDrainNs);
         }
         __syncthreads();
     }
@@ -242,6 +242,149 @@ __global__ void __launch_bounds__(512) centroid_kernel(const uint8_t* kt, uint16
     *reinterpret_cast<uint4*>(cen + ((size_t)b * nblk + j) * row_elems + (size_t)i * 8) = o;
 }
 
+// Fast path for r = 64 and hkv in {4, 8, 16, 32}: warp-specialised pipeline.
+// One producer warp streams 16 KiB chunks through a kQStages-deep ring of TMA
+// bulk copies (full barriers carry the byte count, empty barriers collect one
+// arrival per consumer warp). A consumer warp pass covers 4 tokens x 4 heads:
+// lane = (head-in-quad, token, half-row); each lane keeps its 32 group-sum
+// query values in registers (rotated so that the 8 lanes of a shared-memory
+// phase read 8 distinct 16-byte bank groups), does 32 FMAs, and one shuffle
+// joins the two halves of a row.
+constexpr int kQConsumers = 8;
+constexpr int kQThreads = (kQConsumers + 1) * 32;
+constexpr int kQStages = 6;
+constexpr int kQChunk = 16384;
+
+__global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int hkv = a.hkv;
+    const int token_bytes = hkv * 128;
+    const int tok = a.tok_per_chunk;
+    uint8_t* stages = smem;
+    float* qbar = reinterpret_cast<float*>(smem + kQStages * kQChunk);
+    uint64_t* full = reinterpret_cast<uint64_t*>(qbar + hkv * 64);
+    uint64_t* empty = full + kQStages;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kQStages);
+
+    const int b = blockIdx.y;
+    const int c0 = (int)((long long)blockIdx.x * a.chunks_per_batch / a.ctas_per_batch);
+    const int c1 = (int)((long long)(blockIdx.x + 1) * a.chunks_per_batch / a.ctas_per_batch);
+    const int nch = c1 - c0;
+    const uint8_t* kt_b = a.kt + (size_t)b * a.n * token_bytes;
+
+    for (int e = threadIdx.x; e < hkv * 64; e += kQThreads) {
+        const int h = e >> 6, j = e & 63;
+        const uint16_t* src = a.qt + ((size_t)b * a.hq + (size_t)h * a.G) * 64 + j;
+        float s = 0.f;
+        for (int g = 0; g < a.G; ++g) s += __uint_as_float(((uint32_t)src[(size_t)g * 64]) << 16);
+        qbar[e] = s;
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kQStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kQConsumers);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp == kQConsumers) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < nch; ++i) {
+                const int s = i % kQStages;
+                if (i >= kQStages &&
+                    !mbar_wait_bounded(&empty[s], (uint32_t)(((i / kQStages) - 1) & 1), a.wait_limit, abort_flag)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                const int t0 = (c0 + i) * tok;
+                const int ntok = min(tok, a.n - t0);
+                const uint32_t bytes = (uint32_t)(ntok * token_bytes);
+                mbar_arrive_expect_tx(&full[s], bytes);
+                bulk_g2s(stages + s * kQChunk, kt_b + (size_t)t0 * token_bytes, bytes, &full[s]);
+                issued = i + 1;
+            }
+            if (*abort_flag) {
+                // Leave no bulk copy in flight into this CTA's shared memory.
+                set_status(a.status, kStatusTimeout);
+                for (int s = 0; s < kQStages && s < issued; ++s) {
+                    const int last = s + ((issued - 1 - s) / kQStages) * kQStages;
+                    mbar_wait_bounded(&full[s], (uint32_t)((last / kQStages) & 1), kDrainNs);
+                }
+            }
+        }
+    } else {
+        const int quads = hkv >> 2;
+        const int q = warp % quads;
+        const int wpq = kQConsumers / quads;
+        const int half = lane & 1, tsub = (lane >> 1) & 3, hl = lane >> 3;
+        const int head = q * 4 + hl;
+        float qv[32];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float* src = qbar + head * 64 + half * 32 + ((k + tsub) & 3) * 8;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qv[k * 8 + e] = src[e];
+        }
+        float* out_h = a.out + ((size_t)b * hkv + head) * a.n;
+        for (int i = 0; i < nch; ++i) {
+            const int s = i % kQStages;
+            if (!mbar_wait_bounded(&full[s], (uint32_t)((i / kQStages) & 1), a.wait_limit, abort_flag)) {
+                *abort_flag = 1;
+                break;
+            }
+            const int t0 = (c0 + i) * tok;
+            const int ntok = min(tok, a.n - t0);
+            const uint8_t* st = stages + s * kQChunk + head * 128 + half * 64;
+            for (int tg = warp / quads; tg * 4 < ntok; tg += wpq) {
+                const int t = tg * 4 + tsub;
+                float acc0 = 0.f, acc1 = 0.f;
+                if (t < ntok) {
+                    const uint8_t* row = st + (size_t)t * token_bytes;
+                    const uint4 w0 = *reinterpret_cast<const uint4*>(row + ((0 + tsub) & 3) * 16);
+                    const uint4 w1 = *reinterpret_cast<const uint4*>(row + ((1 + tsub) & 3) * 16);
+                    const uint4 w2 = *reinterpret_cast<const uint4*>(row + ((2 + tsub) & 3) * 16);
+                    const uint4 w3 = *reinterpret_cast<const uint4*>(row + ((3 + tsub) & 3) * 16);
+                    acc0 = dot8(w0, qv + 0);
+                    acc1 = dot8(w1, qv + 8);
+                    acc0 += dot8(w2, qv + 16);
+                    acc1 += dot8(w3, qv + 24);
+                }
+                float acc = acc0 + acc1;
+                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                if (half == 0 && t < ntok) out_h[t0 + t] = finalize_score(acc, a);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+    }
+    __syncthreads();
+}
+
+cudaError_t launch_q64(const LaunchCtx& ctx, ScoreArgs a, int batch) {
+    const int token_bytes = a.hkv * 128;
+    a.tok_per_chunk = kQChunk / token_bytes;
+    a.chunks_per_batch = (a.n + a.tok_per_chunk - 1) / a.tok_per_chunk;
+    const size_t smem = (size_t)kQStages * kQChunk + (size_t)a.hkv * 64 * 4 + 2 * kQStages * 8 + 16;
+    cudaError_t e = ensure_dyn_smem((const void*)score_q64_kernel, (int)smem);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    e = cached_occupancy((const void*)score_q64_kernel, kQThreads, smem, &occ);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) occ = 1;
+    const long long target = (long long)ctx.num_sms * occ;
+    long long per_b = (target + batch - 1) / batch;
+    if (per_b > a.chunks_per_batch) per_b = a.chunks_per_batch;
+    if (per_b < 1) per_b = 1;
+    a.ctas_per_batch = (int)per_b;
+    dim3 grid((unsigned)per_b, (unsigned)batch);
+    score_q64_kernel<<<grid, kQThreads, smem, ctx.stream>>>(a);
+    return cudaGetLastError();
+}
+
 template <int R, bool FIXED>
 cudaError_t launch_flat_t(const LaunchCtx& ctx, ScoreArgs a, int batch) {
     constexpr int LPR = R / 8;
@@ -253,10 +396,10 @@ cudaError_t launch_flat_t(const LaunchCtx& ctx, ScoreArgs a, int batch) {
     a.chunks_per_batch = (a.n + tok - 1) / tok;
     const size_t smem = (size_t)kScoreStages * tok * token_bytes + (size_t)a.hkv * R * 4 + kScoreStages * 8;
     auto kern = score_flat_kernel<R, FIXED>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_dyn_smem((const void*)kern, (int)smem);
     if (e != cudaSuccess) return e;
     int occ = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kScoreThreads, smem);
+    e = cached_occupancy((const void*)kern, kScoreThreads, smem, &occ);
     if (e != cudaSuccess) return e;
     if (occ < 1) occ = 1;
     const long long target = (long long)ctx.num_sms * occ;
@@ -303,6 +446,7 @@ cudaError_t launch_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_
     a.inv_g = 1.0f / (float)a.G;
     a.status = status;
     a.wait_limit = ctx.wait_limit;
+    if (r == 64 && (hkv == 4 || hkv == 8 || hkv == 16 || hkv == 32)) return launch_q64(ctx, a, batch);
     switch (r) {
         case 16: return launch_flat_r<16>(ctx, a, batch);
         case 32: return launch_flat_r<32>(ctx, a, batch);
