@@ -279,15 +279,36 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
         for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
         float L = 0.f;
         if (M != -INFINITY) {
-            for (int s = 0; s < a.nsw; ++s) {
-                const float ms = __ldcg(m + s);
-                if (ms == -INFINITY) continue;
-                const float wgt = exp2f(ms - M);
-                L = fmaf(wgt, __ldcg(l + s), L);
-                const float* o = a.po + (w * a.nsw + s) * D + lane * DPL;
+            // lanes own slots for the weights; the slot loop below keeps eight
+            // independent partial-row loads in flight per lane
+            for (int s0 = 0; s0 < a.nsw; s0 += 32) {
+                const int s = s0 + lane;
+                float wgt = 0.f;
+                if (s < a.nsw) {
+                    const float ms = __ldcg(m + s);
+                    if (ms != -INFINITY) {
+                        wgt = exp2f(ms - M);
+                        L = fmaf(wgt, __ldcg(l + s), L);
+                    }
+                }
+                const int cnt = min(32, a.nsw - s0);
+                for (int j0 = 0; j0 < cnt; j0 += 8) {
+                    float vals[8][DPL];
 #pragma unroll
-                for (int k = 0; k < DPL; ++k) acc[k] = fmaf(wgt, __ldcg(o + k), acc[k]);
+                    for (int u = 0; u < 8; ++u) {
+                        const float* o = a.po + (w * a.nsw + s0 + j0 + u) * D + lane * DPL;
+#pragma unroll
+                        for (int k = 0; k < DPL; ++k) vals[u][k] = j0 + u < cnt ? __ldcg(o + k) : 0.f;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const float wu = __shfl_sync(0xffffffffu, wgt, (j0 + u) & 31);
+#pragma unroll
+                        for (int k = 0; k < DPL; ++k) acc[k] = fmaf(wu, vals[u][k], acc[k]);
+                    }
+                }
             }
+            L = warp_sum(L);
         }
         const float inv = L > 0.f ? 1.f / L : 0.f;
         uint16_t* o = a.out + w * D + lane * DPL;

@@ -72,6 +72,7 @@ struct DecodeLayout {
     size_t idx = 0;           // int32 [batch, hkv, B]
     size_t pm = 0, pl = 0, po = 0;
     size_t counters = 0;      // uint64 [batch, hkv] attention split counters
+    size_t hist = 0;          // uint32 [batch, hkv, 2048] order-key histogram (scorer -> top-B)
     size_t total = 0;
     lsa::AttnPlan plan{};
 };
@@ -102,6 +103,8 @@ DecodeLayout decode_layout(const lsa_dims* d, int B, int blk, int keep, int num_
     off = align_up(off + heads * L.plan.nsw * (size_t)d->d * 4);
     L.counters = off;
     off = align_up(off + units * 8);
+    L.hist = off;
+    off = align_up(off + units * 2048 * 4);
     L.total = off;
     return L;
 }
@@ -220,17 +223,24 @@ lsa_status lsa_decode_step(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf
     const int rows = dims->batch * dims->hkv;
     cudaError_t e;
     if (!hier) {
+        bool hist = false;
+        uint32_t* gh = at<uint32_t>(ws, L.hist);
         e = lsa::launch_score(ctx, qt, kt, at<float>(ws, L.scores), dims->batch, dims->hq, dims->hkv, dims->r, dims->T,
-                              0, status);
-        if (e == cudaSuccess) e = lsa::launch_topk(ctx, at<float>(ws, L.scores), rows, dims->T, B, idx, nullptr, 0, 0);
+                              0, status, gh, &hist);
+        if (e == cudaSuccess)
+            e = lsa::launch_topk(ctx, at<float>(ws, L.scores), rows, dims->T, B, idx, nullptr, 0, 0,
+                                 hist ? gh : nullptr);
     } else {
         const int nblk = (dims->T + blk - 1) / blk;
         int32_t* blkidx = at<int32_t>(ws, L.blkidx);
         float* fine = at<float>(ws, L.fine);
+        bool hist = false;
+        uint32_t* gh = at<uint32_t>(ws, L.hist);
         e = lsa::launch_score(ctx, qt, centroids, at<float>(ws, L.scores), dims->batch, dims->hq, dims->hkv, dims->r,
-                              nblk, 0, status);
+                              nblk, 0, status, gh, &hist);
         if (e == cudaSuccess)
-            e = lsa::launch_topk(ctx, at<float>(ws, L.scores), rows, nblk, nblk_keep, blkidx, nullptr, 0, 0);
+            e = lsa::launch_topk(ctx, at<float>(ws, L.scores), rows, nblk, nblk_keep, blkidx, nullptr, 0, 0,
+                                 hist ? gh : nullptr);
         if (e == cudaSuccess)
             e = lsa::launch_fine_score(ctx, qt, kt, blkidx, nblk_keep, blk, fine, dims->batch, dims->hq, dims->hkv,
                                        dims->r, dims->T);

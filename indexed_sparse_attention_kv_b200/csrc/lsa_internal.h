@@ -60,8 +60,12 @@ struct AttnPlan {
 };
 
 // mode 0: scores are the group-sum dot products (G x the mean); mode 1: means.
+// ghist (optional, [batch * hkv, 2048], zero on entry): the scorer may add the
+// histogram of the top 11 order-key bits of the scores it writes; *hist_done
+// tells whether it did (only some shapes support it).
 cudaError_t launch_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_t* kt, float* out, int batch, int hq,
-                         int hkv, int r, int n, int mode, unsigned* status);
+                         int hkv, int r, int n, int mode, unsigned* status, uint32_t* ghist = nullptr,
+                         bool* hist_done = nullptr);
 
 cudaError_t launch_fine_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_t* kt, const int32_t* blk_idx,
                               int keep, int blk, float* out, int batch, int hq, int hkv, int r, int T);
@@ -69,8 +73,10 @@ cudaError_t launch_fine_score(const LaunchCtx& ctx, const uint16_t* qt, const ui
 cudaError_t launch_centroids(const LaunchCtx& ctx, const uint16_t* kt, int blk, uint16_t* cen, int batch, int hkv, int r,
                              int T);
 
+// ghist (optional): the rows' histograms of key >> 21 from launch_score; the
+// kernel zeroes them after use.
 cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int n, int B, int32_t* idx,
-                        const int32_t* blkmap, int blk, int keep);
+                        const int32_t* blkmap, int blk, int keep, uint32_t* ghist = nullptr);
 
 AttnPlan plan_attn(int nb, int hkv, int G, int B, int num_sms);
 

@@ -34,6 +34,7 @@ struct ScoreArgs {
     float inv_g;
     unsigned* status;
     long long wait_limit;
+    uint32_t* ghist;       // optional [batch, hkv, 2048] key histogram (fast path only)
 };
 
 __device__ __forceinline__ float finalize_score(float acc, const ScoreArgs& a) {
@@ -243,28 +244,34 @@ __global__ void __launch_bounds__(512) centroid_kernel(const uint8_t* kt, uint16
 }
 
 // Fast path for r = 64 and hkv in {4, 8, 16, 32}: warp-specialised pipeline.
-// One producer warp streams 16 KiB chunks through a kQStages-deep ring of TMA
+// One producer warp streams 16 KiB chunks through a STAGES-deep ring of TMA
 // bulk copies (full barriers carry the byte count, empty barriers collect one
 // arrival per consumer warp). A consumer warp pass covers 4 tokens x 4 heads:
 // lane = (head-in-quad, token, half-row); each lane keeps its 32 group-sum
 // query values in registers (rotated so that the 8 lanes of a shared-memory
 // phase read 8 distinct 16-byte bank groups), does 32 FMAs, and one shuffle
 // joins the two halves of a row.
+// HIST: also count, per KV head, the top 11 bits of every score's order key
+// (the first radix digit of the top-B selection) in a shared-memory histogram
+// of 16-bit counters, added to a global per-(sequence, head) histogram at the
+// end; that saves the selection a full pass over the scores.
 constexpr int kQConsumers = 8;
 constexpr int kQThreads = (kQConsumers + 1) * 32;
-constexpr int kQStages = 6;
 constexpr int kQChunk = 16384;
+constexpr int kHistBins = 2048;
 
+template <int STAGES, bool HIST>
 __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int hkv = a.hkv;
     const int token_bytes = hkv * 128;
     const int tok = a.tok_per_chunk;
     uint8_t* stages = smem;
-    float* qbar = reinterpret_cast<float*>(smem + kQStages * kQChunk);
-    uint64_t* full = reinterpret_cast<uint64_t*>(qbar + hkv * 64);
-    uint64_t* empty = full + kQStages;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kQStages);
+    float* qbar = reinterpret_cast<float*>(smem + STAGES * kQChunk);
+    uint32_t* hs = reinterpret_cast<uint32_t*>(qbar + hkv * 64);          // [hkv][kHistBins / 2] (HIST)
+    uint64_t* full = reinterpret_cast<uint64_t*>(hs + (HIST ? hkv * kHistBins / 2 : 0));
+    uint64_t* empty = full + STAGES;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + STAGES);
 
     const int b = blockIdx.y;
     const int c0 = (int)((long long)blockIdx.x * a.chunks_per_batch / a.ctas_per_batch);
@@ -279,8 +286,10 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
         for (int g = 0; g < a.G; ++g) s += __uint_as_float(((uint32_t)src[(size_t)g * 64]) << 16);
         qbar[e] = s;
     }
+    if (HIST)
+        for (int e = threadIdx.x; e < hkv * kHistBins / 2; e += kQThreads) hs[e] = 0u;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kQStages; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kQConsumers);
         }
@@ -294,9 +303,9 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
         if (lane == 0) {
             int issued = 0;
             for (int i = 0; i < nch; ++i) {
-                const int s = i % kQStages;
-                if (i >= kQStages &&
-                    !mbar_wait_bounded(&empty[s], (uint32_t)(((i / kQStages) - 1) & 1), a.wait_limit, abort_flag)) {
+                const int s = i % STAGES;
+                if (i >= STAGES &&
+                    !mbar_wait_bounded(&empty[s], (uint32_t)(((i / STAGES) - 1) & 1), a.wait_limit, abort_flag)) {
                     *abort_flag = 1;
                     break;
                 }
@@ -310,9 +319,9 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
             if (*abort_flag) {
                 // Leave no bulk copy in flight into this CTA's shared memory.
                 set_status(a.status, kStatusTimeout);
-                for (int s = 0; s < kQStages && s < issued; ++s) {
-                    const int last = s + ((issued - 1 - s) / kQStages) * kQStages;
-                    mbar_wait_bounded(&full[s], (uint32_t)((last / kQStages) & 1), kDrainNs);
+                for (int s = 0; s < STAGES && s < issued; ++s) {
+                    const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
+                    mbar_wait_bounded(&full[s], (uint32_t)((last / STAGES) & 1), kDrainNs);
                 }
             }
         }
@@ -330,9 +339,10 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
             for (int e = 0; e < 8; ++e) qv[k * 8 + e] = src[e];
         }
         float* out_h = a.out + ((size_t)b * hkv + head) * a.n;
+        uint32_t* hs_h = hs + head * (kHistBins / 2);
         for (int i = 0; i < nch; ++i) {
-            const int s = i % kQStages;
-            if (!mbar_wait_bounded(&full[s], (uint32_t)((i / kQStages) & 1), a.wait_limit, abort_flag)) {
+            const int s = i % STAGES;
+            if (!mbar_wait_bounded(&full[s], (uint32_t)((i / STAGES) & 1), a.wait_limit, abort_flag)) {
                 *abort_flag = 1;
                 break;
             }
@@ -355,24 +365,42 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
                 }
                 float acc = acc0 + acc1;
                 acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                if (half == 0 && t < ntok) out_h[t0 + t] = finalize_score(acc, a);
+                if (half == 0 && t < ntok) {
+                    const float v = finalize_score(acc, a);
+                    out_h[t0 + t] = v;
+                    if (HIST) {
+                        const uint32_t key = score_key(v);
+                        if (key) atomicAdd(&hs_h[key >> 22], 1u << (((key >> 21) & 1u) * 16));
+                    }
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
     }
     __syncthreads();
+    if (HIST) {
+        uint32_t* gh = a.ghist + (size_t)b * hkv * kHistBins;
+        for (int e = threadIdx.x; e < hkv * kHistBins / 2; e += kQThreads) {
+            const uint32_t v = hs[e];
+            if (!v) continue;
+            const int h = e / (kHistBins / 2), w = e - h * (kHistBins / 2);
+            uint32_t* dst = gh + (size_t)h * kHistBins + 2 * w;
+            if (v & 0xffffu) atomicAdd(dst, v & 0xffffu);
+            if (v >> 16) atomicAdd(dst + 1, v >> 16);
+        }
+    }
 }
 
-cudaError_t launch_q64(const LaunchCtx& ctx, ScoreArgs a, int batch) {
-    const int token_bytes = a.hkv * 128;
-    a.tok_per_chunk = kQChunk / token_bytes;
-    a.chunks_per_batch = (a.n + a.tok_per_chunk - 1) / a.tok_per_chunk;
-    const size_t smem = (size_t)kQStages * kQChunk + (size_t)a.hkv * 64 * 4 + 2 * kQStages * 8 + 16;
-    cudaError_t e = ensure_dyn_smem((const void*)score_q64_kernel, (int)smem);
+template <int STAGES, bool HIST>
+cudaError_t launch_q64_t(const LaunchCtx& ctx, ScoreArgs a, int batch) {
+    const size_t smem = (size_t)STAGES * kQChunk + (size_t)a.hkv * 64 * 4 +
+                        (HIST ? (size_t)a.hkv * kHistBins / 2 * 4 : 0) + 2 * STAGES * 8 + 16;
+    auto kern = score_q64_kernel<STAGES, HIST>;
+    cudaError_t e = ensure_dyn_smem((const void*)kern, (int)smem);
     if (e != cudaSuccess) return e;
     int occ = 0;
-    e = cached_occupancy((const void*)score_q64_kernel, kQThreads, smem, &occ);
+    e = cached_occupancy((const void*)kern, kQThreads, smem, &occ);
     if (e != cudaSuccess) return e;
     if (occ < 1) occ = 1;
     const long long target = (long long)ctx.num_sms * occ;
@@ -381,8 +409,26 @@ cudaError_t launch_q64(const LaunchCtx& ctx, ScoreArgs a, int batch) {
     if (per_b < 1) per_b = 1;
     a.ctas_per_batch = (int)per_b;
     dim3 grid((unsigned)per_b, (unsigned)batch);
-    score_q64_kernel<<<grid, kQThreads, smem, ctx.stream>>>(a);
+    kern<<<grid, kQThreads, smem, ctx.stream>>>(a);
     return cudaGetLastError();
+}
+
+// Returns whether the histogram was produced (a.ghist non-null, hkv <= 8 and at
+// most 65535 tokens per CTA so that 16-bit shared counters cannot overflow).
+cudaError_t launch_q64(const LaunchCtx& ctx, ScoreArgs a, int batch, bool* hist_done) {
+    const int token_bytes = a.hkv * 128;
+    a.tok_per_chunk = kQChunk / token_bytes;
+    a.chunks_per_batch = (a.n + a.tok_per_chunk - 1) / a.tok_per_chunk;
+    bool hist = a.ghist != nullptr && a.hkv <= 8;
+    if (hist) {
+        // the smallest grid the launcher can pick: one CTA per SM (occupancy >= 1)
+        const long long min_per_b = ((long long)ctx.num_sms + batch - 1) / batch;
+        const long long per_b = min_per_b < a.chunks_per_batch ? min_per_b : a.chunks_per_batch;
+        const long long max_chunks = (a.chunks_per_batch + per_b - 1) / per_b;
+        hist = max_chunks * a.tok_per_chunk <= 65535;
+    }
+    *hist_done = hist;
+    return hist ? launch_q64_t<4, true>(ctx, a, batch) : launch_q64_t<6, false>(ctx, a, batch);
 }
 
 template <int R, bool FIXED>
@@ -432,7 +478,7 @@ cudaError_t launch_fine_r(const LaunchCtx& ctx, const FineArgs& a, int batch) {
 }  // namespace
 
 cudaError_t launch_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_t* kt, float* out, int batch, int hq,
-                         int hkv, int r, int n, int mode, unsigned* status) {
+                         int hkv, int r, int n, int mode, unsigned* status, uint32_t* ghist, bool* hist_done) {
     ScoreArgs a{};
     a.qt = qt;
     a.kt = reinterpret_cast<const uint8_t*>(kt);
@@ -446,7 +492,11 @@ cudaError_t launch_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_
     a.inv_g = 1.0f / (float)a.G;
     a.status = status;
     a.wait_limit = ctx.wait_limit;
-    if (r == 64 && (hkv == 4 || hkv == 8 || hkv == 16 || hkv == 32)) return launch_q64(ctx, a, batch);
+    a.ghist = ghist;
+    if (hist_done) *hist_done = false;
+    bool dummy = false;
+    if (r == 64 && (hkv == 4 || hkv == 8 || hkv == 16 || hkv == 32))
+        return launch_q64(ctx, a, batch, hist_done ? hist_done : &dummy);
     switch (r) {
         case 16: return launch_flat_r<16>(ctx, a, batch);
         case 32: return launch_flat_r<32>(ctx, a, batch);

@@ -5,18 +5,25 @@
 // the threshold go to the lower position; the set is written in ascending order
 // and padded with -1 when fewer than B candidates (non-NaN scores) exist.
 //
-// One cluster of CS CTAs owns a row; CTA k owns a contiguous segment of it.
-// Scores map to order-preserving 32-bit keys (NaN -> 0, never selected).
-//   1. histogram of the top 11 key bits (warp-aggregated shared atomics);
-//      every CTA sums the cluster's histograms through distributed shared
-//      memory and finds the bin b0 that holds the B-th largest key;
-//   2. every CTA collects its keys that fall in b0; when the cluster holds few
-//      of them, every CTA gathers all of them and resolves the exact threshold
-//      key theta (and how many ties at theta to take) with two local radix
-//      passes; otherwise two more cluster-wide radix passes do it;
-//   3. per-warp counts of keys above / equal to theta, exclusive prefix sums
-//      over warps and over the cluster's CTAs, and a compaction pass with warp
-//      ballots in position order write the selected positions ascending.
+// Scores map to order-preserving 32-bit keys (NaN -> 0, never selected). One
+// cluster of CS CTAs owns a row, CTA k a contiguous segment of it, warp w of a
+// CTA a contiguous sub-range of that segment.
+//   1. The histogram of the top 11 key bits of the whole row: either built by
+//      the scorer while it wrote the scores (decode path), or here, per CTA in
+//      shared memory and summed over the cluster through distributed shared
+//      memory. From it, the bin b0 holding the B-th largest key.
+//   2. One pass over the keys in position order: every warp appends the
+//      (key, position) pairs of bin >= b0 to its own list (about B plus the
+//      threshold bin's keys per row: a small fraction of the row).
+//   3. The keys of bin b0 of the whole cluster are gathered in every CTA and two
+//      local radix passes give the exact threshold key theta and the number of
+//      ties at theta to take.
+//   4. Counts above / at theta per warp, exclusive prefix sums over warps and
+//      over the cluster's CTAs, and a ballot compaction of the short lists write
+//      the positions in ascending order.
+// Whenever a list or the threshold bin is too large for shared memory (e.g.
+// many equal scores), the cluster switches, uniformly, to radix passes and a
+// compaction over the keys themselves, with the same result.
 #include <cooperative_groups.h>
 
 #include "lsa_common.cuh"
@@ -30,33 +37,32 @@ namespace {
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kSegCap = 16384;     // keys staged in shared memory per CTA (64 KiB)
 constexpr int kBins = 2048;
-constexpr int kCandCap = 4096;     // threshold-bin keys kept per CTA
-constexpr int kGatherCap = 4096;   // threshold-bin keys gathered from the whole cluster
+constexpr int kListPerWarp = 256;                       // (key, position) entries per warp
+constexpr int kListCap = kListPerWarp * kTopkWarps;     // per CTA
+constexpr int kGatherCap = 4096;                        // bin-b0 keys of the whole cluster
 constexpr int kMaxCluster = 8;
 
 struct TopkArgs {
     const float* scores;      // [rows, n]
     int32_t* idx;             // [rows, B]
     const int32_t* blkmap;    // optional [rows, keep]: candidate c -> blkmap[c / blk] * blk + c % blk
-    int n, B, seg, staged, blk, keep;
+    uint32_t* ghist;          // optional [rows, kBins] histogram of key >> 21; zeroed here after use
+    int n, B, seg, blk, keep;
 };
 
 struct TopkShared {
-    union {
-        struct {
-            uint32_t hist[kBins];
-            uint32_t red[kBins];
-        } h;
-        uint32_t gathered[kGatherCap];
-    } u;
-    uint32_t lhist[kBins];
-    uint32_t cand[kCandCap];
+    uint32_t red[kBins];            // row histogram
+    uint32_t hist[kBins];           // this CTA's histogram / local refinement histogram
+    uint32_t lkey[kListCap];        // per-warp lists (position order) of keys in bins >= b0
+    int lpos[kListCap];
+    uint32_t cand[kListCap];        // this CTA's bin-b0 keys (any order)
+    uint32_t gathered[kGatherCap];  // the cluster's bin-b0 keys
+    int wlist[kTopkWarps], wb0[kTopkWarps];
     int scan[kTopkWarps];
     int warp_gt[kTopkWarps], warp_eq[kTopkWarps];
     int warp_sel_before[kTopkWarps], warp_eq_before[kTopkWarps];
-    int cta_gt, cta_eq, ncand;
+    int cta_gt, cta_eq, ncand, overflow;
     uint32_t bstar;
     int above;
     int total;
@@ -91,6 +97,19 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scan, int* total) {
     return res;
 }
 
+// Warp-level exclusive prefix sum; *total = the warp's sum.
+__device__ __forceinline__ int warp_excl_scan(int v, int* total) {
+    const int lane = threadIdx.x & 31;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    *total = __shfl_sync(0xffffffffu, x, 31);
+    return x - v;
+}
+
 // Given histogram `red` (nb bins) find the bin holding the krem-th largest
 // element counted from the top; sets sh.bstar and sh.above (count above it)
 // and returns the histogram total. All threads must call it.
@@ -117,145 +136,243 @@ __device__ __forceinline__ int find_bin(const uint32_t* red, int nb, int krem, T
     return total;
 }
 
-// Warp-aggregated histogram increment: lanes with equal bins add once.
-__device__ __forceinline__ void hist_add(uint32_t* h, bool active, uint32_t bin) {
-    const uint32_t key = active ? bin : 0xffffffffu;
-    const unsigned peers = __match_any_sync(0xffffffffu, key);
-    const int leader = __ffs(peers) - 1;
-    if (active && (int)(threadIdx.x & 31) == leader) atomicAdd(&h[bin], (uint32_t)__popc(peers));
-}
-
-// Sum histogram `h` (nb bins) over the cluster's CTAs into `red`.
+// Sum histogram `h` (nb <= kBins bins) over the cluster's CTAs into `red`; all
+// of a thread's remote loads are independent and in flight together.
 __device__ __forceinline__ void cluster_reduce(cg::cluster_group& cluster, uint32_t* h, uint32_t* red, int nb, int CS) {
-    for (int bin = threadIdx.x; bin < nb; bin += kTopkThreads) {
-        uint32_t v[kMaxCluster];
+    constexpr int kPer = kBins / kTopkThreads;
+    uint32_t v[kPer][kMaxCluster];
 #pragma unroll
-        for (int rr = 0; rr < kMaxCluster; ++rr) v[rr] = rr < CS ? cluster.map_shared_rank(h, rr)[bin] : 0u;
+    for (int q = 0; q < kPer; ++q) {
+        const int bin = q * kTopkThreads + threadIdx.x;
+#pragma unroll
+        for (int rr = 0; rr < kMaxCluster; ++rr)
+            v[q][rr] = (rr < CS && bin < nb) ? cluster.map_shared_rank(h, rr)[bin] : 0u;
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int bin = q * kTopkThreads + threadIdx.x;
         uint32_t s = 0;
 #pragma unroll
-        for (int rr = 0; rr < kMaxCluster; ++rr) s += v[rr];
-        red[bin] = s;
+        for (int rr = 0; rr < kMaxCluster; ++rr) s += v[q][rr];
+        if (bin < nb) red[bin] = s;
     }
 }
 
+// The 4 keys at sub-range positions i .. i+3 (i a multiple of 4) of a warp
+// range ending at `end`; 16-byte loads when the row is 16-byte aligned.
+__device__ __forceinline__ void load4(const float* src, bool vec, int i, int end, uint32_t k[4]) {
+    if (vec && i + 3 < end) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(src + i));
+        k[0] = score_key(v.x);
+        k[1] = score_key(v.y);
+        k[2] = score_key(v.z);
+        k[3] = score_key(v.w);
+    } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) k[u] = i + u < end ? score_key(__ldcg(src + i + u)) : 0u;
+    }
+}
+
+template <bool EXT_HIST>
 __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkArgs a) {
     cg::cluster_group cluster = cg::this_cluster();
     const int CS = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
     const int row = blockIdx.y;
-    __shared__ TopkShared sh;
-    extern __shared__ uint32_t keys[];
+    extern __shared__ __align__(16) uint8_t topk_smem[];
+    TopkShared& sh = *reinterpret_cast<TopkShared*>(topk_smem);
 
     const int base = rank * a.seg;
     int len = a.n - base;
     len = len < 0 ? 0 : (len > a.seg ? a.seg : len);
     const float* src = a.scores + (size_t)row * a.n + base;
+    const bool vec = (a.n & 3) == 0;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // warp sub-range of the segment, a multiple of 128 keys (4 per lane per step)
+    int wlen = (len + kTopkWarps - 1) / kTopkWarps;
+    wlen = (wlen + 127) & ~127;
+    const int wbeg = min(len, warp * wlen), wend = min(len, wbeg + wlen);
 
-    if (a.staged)
-        for (int i = tid; i < len; i += kTopkThreads) keys[i] = score_key(src[i]);
-    auto key_at = [&](int i) -> uint32_t { return a.staged ? keys[i] : score_key(src[i]); };
-    const int len_up = (len + 31) & ~31;
-
-    // ---- 1. top-11-bit histogram, cluster sum, threshold bin b0
-    for (int i = tid; i < kBins; i += kTopkThreads) sh.u.h.hist[i] = 0;
-    if (tid == 0) sh.ncand = 0;
-    __syncthreads();
-    for (int i = tid; i < len_up; i += kTopkThreads) {
-        const uint32_t k = i < len ? key_at(i) : 0u;
-        hist_add(sh.u.h.hist, k != 0u, k >> 21);
-    }
-    cluster.sync();
-    cluster_reduce(cluster, sh.u.h.hist, sh.u.h.red, kBins, CS);
-    __syncthreads();
-    int krem = a.B;
-    const int total = find_bin(sh.u.h.red, kBins, krem, sh);
-    const bool take_all = total <= a.B;
-    uint32_t theta = 0;
-    if (!take_all) {
-        const uint32_t b0 = sh.bstar;
-        krem -= sh.above;
-        const int in_b0 = (int)sh.u.h.red[b0];
-        // ---- 2. collect this CTA's keys in b0
-        for (int i = tid; i < len_up; i += kTopkThreads) {
-            const uint32_t k = i < len ? key_at(i) : 0u;
-            const bool hit = k != 0u && (k >> 21) == b0;
-            const unsigned m = __ballot_sync(0xffffffffu, hit);
-            int off = 0;
-            if (lane == 0 && m) off = atomicAdd(&sh.ncand, __popc(m));
-            off = __shfl_sync(0xffffffffu, off, 0);
-            const int slot = off + __popc(m & ((1u << lane) - 1u));
-            if (hit && slot < kCandCap) sh.cand[slot] = k;
+    // ---- 1. row histogram of key >> 21 and the threshold bin b0
+    if (EXT_HIST) {
+        for (int i = tid; i < kBins; i += kTopkThreads) sh.red[i] = a.ghist[(size_t)row * kBins + i];
+        __syncthreads();
+    } else {
+        for (int i = tid; i < kBins; i += kTopkThreads) sh.hist[i] = 0;
+        __syncthreads();
+        for (int i0 = wbeg; i0 < wend; i0 += 128) {
+            uint32_t k[4];
+            load4(src, vec, i0 + lane * 4, wend, k);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (k[u]) atomicAdd(&sh.hist[k[u] >> 21], 1u);
         }
-        cluster.sync();   // every CTA's hist/red reads are done; candidate lists complete
-        const bool local_ok = in_b0 <= kGatherCap;
-        if (local_ok) {
-            // gather the cluster's b0 keys (rank order), then two local radix passes
-            int off = 0;
-            for (int rr = 0; rr < CS; ++rr) {
-                const TopkShared* o = cluster.map_shared_rank(&sh, rr);
-                const int nc = min(o->ncand, kCandCap);
-                for (int i = tid; i < nc; i += kTopkThreads) sh.u.gathered[off + i] = o->cand[i];
-                off += nc;
+        cluster.sync();
+        cluster_reduce(cluster, sh.hist, sh.red, kBins, CS);
+        __syncthreads();
+    }
+    int krem = a.B;
+    const int total = find_bin(sh.red, kBins, krem, sh);
+    const bool take_all = total <= a.B;
+    const uint32_t b0 = take_all ? 0u : sh.bstar;
+    if (!take_all) krem -= sh.above;
+    const int in_b0 = take_all ? 0 : (int)sh.red[b0];
+
+    // ---- 2. per-warp lists of (key, position) with bin >= b0, in position order
+    uint32_t* wkey = sh.lkey + warp * kListPerWarp;
+    int* wpos = sh.lpos + warp * kListPerWarp;
+    int wc = 0;
+    for (int i0 = wbeg; i0 < wend; i0 += 128) {
+        const int i = i0 + lane * 4;
+        uint32_t k[4];
+        load4(src, vec, i, wend, k);
+        bool f[4];
+        int c = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            f[u] = k[u] != 0u && (k[u] >> 21) >= b0;
+            c += f[u];
+        }
+        int tot;
+        int slot = wc + warp_excl_scan(c, &tot);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (f[u]) {
+                if (slot < kListPerWarp) {
+                    wkey[slot] = k[u];
+                    wpos[slot] = base + i + u;
+                }
+                ++slot;
+            }
+        }
+        wc += tot;
+    }
+    if (lane == 0) sh.wlist[warp] = wc;
+    __syncthreads();
+    bool over = false;
+    for (int w = 0; w < kTopkWarps; ++w) over |= sh.wlist[w] > kListPerWarp;
+    if (!take_all && !over) {
+        // pack this CTA's bin-b0 keys for the cluster gather
+        int nb0 = 0;
+        for (int j = lane; j < ((wc + 31) & ~31); j += 32) {
+            const bool hit = j < wc && (wkey[j] >> 21) == b0;
+            nb0 += __popc(__ballot_sync(0xffffffffu, hit));
+        }
+        if (lane == 0) sh.wb0[warp] = nb0;
+        __syncthreads();
+        int off = 0;
+        for (int w = 0; w < warp; ++w) off += sh.wb0[w];
+        for (int j0 = 0; j0 < wc; j0 += 32) {
+            const int j = j0 + lane;
+            const bool hit = j < wc && (wkey[j] >> 21) == b0;
+            const unsigned m = __ballot_sync(0xffffffffu, hit);
+            if (hit) sh.cand[off + __popc(m & ((1u << lane) - 1u))] = wkey[j];
+            off += __popc(m);
+        }
+        if (tid == 0) {
+            int t = 0;
+            for (int w = 0; w < kTopkWarps; ++w) t += sh.wb0[w];
+            sh.ncand = t;
+        }
+    }
+    if (tid == 0) sh.overflow = over;
+    cluster.sync();   // lists, packed keys and flags complete; every CTA has read the row histogram
+    if (EXT_HIST && rank == 0)
+        for (int i = tid; i < kBins; i += kTopkThreads) a.ghist[(size_t)row * kBins + i] = 0u;
+    int any_over = 0;
+#pragma unroll
+    for (int rr = 0; rr < kMaxCluster; ++rr) any_over |= rr < CS ? cluster.map_shared_rank(&sh, rr)->overflow : 0;
+
+    // ---- 3. exact threshold theta and the ties at theta to take
+    uint32_t theta = 0;
+    int cnt[kMaxCluster];
+    int ncand_all = 0;
+#pragma unroll
+    for (int rr = 0; rr < kMaxCluster; ++rr) {
+        cnt[rr] = (rr < CS && !take_all && !any_over) ? cluster.map_shared_rank(&sh, rr)->ncand : 0;
+        ncand_all += cnt[rr];
+    }
+    // the packed counts, not the histogram, decide: the gather can never overrun
+    const bool local_ok = !take_all && !any_over && ncand_all <= kGatherCap;
+    (void)in_b0;
+    if (local_ok) {
+        int off = 0;
+#pragma unroll
+        for (int rr = 0; rr < kMaxCluster; ++rr) {
+            if (rr < CS) {
+                const uint32_t* c = cluster.map_shared_rank(sh.cand, rr);
+                for (int i = tid; i < cnt[rr]; i += kTopkThreads) sh.gathered[off + i] = c[i];
+            }
+            off += cnt[rr];
+        }
+        __syncthreads();
+        uint32_t prefix = b0 << 21, pmask = 0xffe00000u;
+        for (int pass = 1; pass < 3; ++pass) {
+            const int shift = pass == 1 ? 10 : 0;
+            const int nb = pass == 1 ? 2048 : 1024;
+            for (int i = tid; i < nb; i += kTopkThreads) sh.hist[i] = 0;
+            __syncthreads();
+            for (int i = tid; i < off; i += kTopkThreads) {
+                const uint32_t k = sh.gathered[i];
+                if ((k & pmask) == prefix) atomicAdd(&sh.hist[(k >> shift) & (uint32_t)(nb - 1)], 1u);
             }
             __syncthreads();
-            uint32_t prefix = b0 << 21, pmask = 0xffe00000u;
-            for (int pass = 1; pass < 3; ++pass) {
-                const int shift = pass == 1 ? 10 : 0;
-                const int nb = pass == 1 ? 2048 : 1024;
-                for (int i = tid; i < nb; i += kTopkThreads) sh.lhist[i] = 0;
-                __syncthreads();
-                for (int i = tid; i < ((off + 31) & ~31); i += kTopkThreads) {
-                    const uint32_t k = i < off ? sh.u.gathered[i] : 0u;
-                    hist_add(sh.lhist, i < off && (k & pmask) == prefix, (k >> shift) & (uint32_t)(nb - 1));
-                }
-                __syncthreads();
-                find_bin(sh.lhist, nb, krem, sh);
-                prefix |= sh.bstar << shift;
-                pmask |= (uint32_t)(nb - 1) << shift;
-                krem -= sh.above;
-                __syncthreads();
-            }
-            theta = prefix;
+            find_bin(sh.hist, nb, krem, sh);
+            prefix |= sh.bstar << shift;
+            pmask |= (uint32_t)(nb - 1) << shift;
+            krem -= sh.above;
+            __syncthreads();
         }
-        cluster.sync();   // remote readers of cand / ncand are done
-        if (!local_ok) {
-            // many keys share b0: resolve the low 21 bits with cluster-wide passes
-            uint32_t prefix = b0 << 21, pmask = 0xffe00000u;
-            for (int pass = 1; pass < 3; ++pass) {
-                const int shift = pass == 1 ? 10 : 0;
-                const int nb = pass == 1 ? 2048 : 1024;
-                uint32_t* h = sh.lhist;
-                for (int i = tid; i < nb; i += kTopkThreads) h[i] = 0;
-                __syncthreads();
-                for (int i = tid; i < len_up; i += kTopkThreads) {
-                    const uint32_t k = i < len ? key_at(i) : 0u;
-                    hist_add(h, k != 0u && (k & pmask) == prefix, (k >> shift) & (uint32_t)(nb - 1));
-                }
-                cluster.sync();
-                cluster_reduce(cluster, h, sh.u.h.red, nb, CS);
-                cluster.sync();   // lhist may be reset next pass only after every CTA has read it
-                find_bin(sh.u.h.red, nb, krem, sh);
-                prefix |= sh.bstar << shift;
-                pmask |= (uint32_t)(nb - 1) << shift;
-                krem -= sh.above;
-                __syncthreads();
+        theta = prefix;
+    }
+    cluster.sync();   // remote reads of the packed keys are done
+    if (!take_all && !local_ok) {
+        // too many keys for shared memory: resolve the low 21 bits with
+        // cluster-wide radix passes over the keys themselves
+        uint32_t prefix = b0 << 21, pmask = 0xffe00000u;
+        for (int pass = 1; pass < 3; ++pass) {
+            const int shift = pass == 1 ? 10 : 0;
+            const int nb = pass == 1 ? 2048 : 1024;
+            for (int i = tid; i < nb; i += kTopkThreads) sh.hist[i] = 0;
+            __syncthreads();
+            for (int i0 = wbeg; i0 < wend; i0 += 128) {
+                uint32_t k[4];
+                load4(src, vec, i0 + lane * 4, wend, k);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (k[u] && (k[u] & pmask) == prefix) atomicAdd(&sh.hist[(k[u] >> shift) & (uint32_t)(nb - 1)], 1u);
             }
-            theta = prefix;
+            cluster.sync();
+            cluster_reduce(cluster, sh.hist, sh.red, nb, CS);
+            cluster.sync();   // hist may be reset next pass only after every CTA has read it
+            find_bin(sh.red, nb, krem, sh);
+            prefix |= sh.bstar << shift;
+            pmask |= (uint32_t)(nb - 1) << shift;
+            krem -= sh.above;
+            __syncthreads();
+        }
+        theta = prefix;
+    }
+    if (take_all) krem = 0;   // every valid key (key > 0 = theta) is taken
+
+    // ---- 4. counts per warp (position order), offsets, compaction
+    int gt = 0, eq = 0;
+    if (!any_over) {
+        for (int j = lane; j < wc; j += 32) {
+            const uint32_t k = wkey[j];
+            gt += k > theta;
+            eq += k == theta;
         }
     } else {
-        krem = 0;   // every candidate (key > 0) is selected
-    }
-
-    // ---- 3. counts per warp over contiguous warp ranges (position order)
-    int wlen = (len + kTopkWarps - 1) / kTopkWarps;
-    wlen = (wlen + 31) & ~31;
-    const int wbeg = min(len, warp * wlen), wend = min(len, wbeg + wlen);
-    int gt = 0, eq = 0;
-    for (int i = wbeg + lane; i < wend; i += 32) {
-        const uint32_t k = key_at(i);
-        gt += k > theta;
-        eq += k == theta;
+        for (int i0 = wbeg; i0 < wend; i0 += 128) {
+            uint32_t k[4];
+            load4(src, vec, i0 + lane * 4, wend, k);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                gt += k[u] > theta;
+                eq += k[u] == theta && i0 + lane * 4 + u < wend;
+            }
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -278,18 +395,25 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkAr
     }
     cluster.sync();
     if (tid == 0) {
-        // Tie quota and output offset of every CTA, in rank (= position) order.
+        // tie quota and output offset of every CTA, in rank (= position) order
+        int cgt[kMaxCluster], ceq[kMaxCluster];
+#pragma unroll
+        for (int rr = 0; rr < kMaxCluster; ++rr) {
+            const TopkShared* o = cluster.map_shared_rank(&sh, rr < CS ? rr : 0);
+            cgt[rr] = rr < CS ? o->cta_gt : 0;
+            ceq[rr] = rr < CS ? o->cta_eq : 0;
+        }
         int eq_before = 0, sel_before = 0, eq_run = 0, sel_total = 0;
-        for (int rr = 0; rr < CS; ++rr) {
-            const TopkShared* o = cluster.map_shared_rank(&sh, rr);
+#pragma unroll
+        for (int rr = 0; rr < kMaxCluster; ++rr) {
             int take = krem - eq_run;
-            take = take < 0 ? 0 : (take > o->cta_eq ? o->cta_eq : take);
+            take = take < 0 ? 0 : (take > ceq[rr] ? ceq[rr] : take);
             if (rr == rank) {
                 eq_before = eq_run;
                 sel_before = sel_total;
             }
-            eq_run += o->cta_eq;
-            sel_total += o->cta_gt + take;
+            eq_run += ceq[rr];
+            sel_total += cgt[rr] + take;
         }
         int e = eq_before, s = sel_before;
         for (int w = 0; w < kTopkWarps; ++w) {
@@ -304,33 +428,42 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkAr
     }
     __syncthreads();
 
-    // ---- compaction in position order
     int32_t* out = a.idx + (size_t)row * a.B;
     const int32_t* bm = a.blkmap ? a.blkmap + (size_t)row * a.keep : nullptr;
     const int eq_before = sh.warp_eq_before[warp];
     int sel_pos = sh.warp_sel_before[warp];
     int eq_seen = 0;
     const unsigned lt_mask = (1u << lane) - 1u;
-    for (int i0 = wbeg; i0 < wend; i0 += 32) {
-        const int i = i0 + lane;
-        const bool in = i < wend;
-        const uint32_t k = in ? key_at(i) : 0u;
+    auto emit = [&](bool in, uint32_t k, int c) {
         const bool is_eq = in && k == theta;
         const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
         const int rank_eq = eq_before + eq_seen + __popc(eqm & lt_mask);
         const bool take = in && (k > theta || (is_eq && rank_eq < krem));
         const unsigned sm = __ballot_sync(0xffffffffu, take);
-        if (take) {
-            const int c = base + i;
+        const int dst = sel_pos + __popc(sm & lt_mask);
+        if (take && dst < a.B) {   // always true for a consistent histogram; never writes past B
             int pos = c;
             if (bm) {
                 const int j = c / a.blk;
                 pos = bm[j] * a.blk + (c - j * a.blk);
             }
-            out[sel_pos + __popc(sm & lt_mask)] = pos;
+            out[dst] = pos;
         }
         eq_seen += __popc(eqm);
         sel_pos += __popc(sm);
+    };
+    if (!any_over) {
+        for (int j0 = 0; j0 < wc; j0 += 32) {
+            const int j = j0 + lane;
+            const bool in = j < wc;
+            emit(in, in ? wkey[j] : 0u, in ? wpos[j] : 0);
+        }
+    } else {
+        for (int i0 = wbeg; i0 < wend; i0 += 32) {
+            const int i = i0 + lane;
+            const bool in = i < wend;
+            emit(in, in ? score_key(__ldcg(src + i)) : 0u, base + i);
+        }
     }
     if (rank == CS - 1)
         for (int p = sh.total + tid; p < a.B; p += kTopkThreads) out[p] = -1;
@@ -340,31 +473,32 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkAr
 }  // namespace
 
 cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int n, int B, int32_t* idx,
-                        const int32_t* blkmap, int blk, int keep) {
+                        const int32_t* blkmap, int blk, int keep, uint32_t* ghist) {
     TopkArgs a{};
     a.scores = scores;
     a.idx = idx;
     a.blkmap = blkmap;
+    a.ghist = ghist;
     a.n = n;
     a.B = B;
     a.blk = blk;
     a.keep = keep;
-    // Cluster size: enough CTAs to spread the row, at most 8 (portable).
+    // Cluster size: about 16K keys per CTA, at most 8 (portable); fewer CTAs
+    // per row when there are many rows.
     int cs = 1;
-    while (cs < kMaxCluster && (long long)cs * 4096 < n) cs <<= 1;
-    // Prefer fewer CTAs per row when there are many rows.
-    while (cs > 1 && (long long)rows * cs > 4ll * ctx.num_sms && (n + cs / 2 - 1) / (cs / 2) <= kSegCap) cs >>= 1;
+    while (cs < kMaxCluster && (long long)cs * 16384 < n) cs <<= 1;
+    while (cs < kMaxCluster && (long long)rows * cs * 2 <= 2ll * ctx.num_sms && (long long)cs * 4096 < n) cs <<= 1;
     int seg = (n + cs - 1) / cs;
-    seg = (seg + 31) & ~31;
+    seg = (seg + 127) & ~127;
     a.seg = seg;
-    a.staged = seg <= kSegCap;
-    const size_t dyn = a.staged ? (size_t)seg * 4 : 0;
-    cudaError_t e = ensure_dyn_smem((const void*)topk_cluster_kernel, (int)(kSegCap * 4));
+    const size_t smem = sizeof(TopkShared);
+    auto kern = ghist ? topk_cluster_kernel<true> : topk_cluster_kernel<false>;
+    cudaError_t e = ensure_dyn_smem((const void*)kern, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)cs, (unsigned)rows);
     cfg.blockDim = dim3(kTopkThreads);
-    cfg.dynamicSmemBytes = dyn;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = ctx.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -373,7 +507,7 @@ cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, a);
+    e = cudaLaunchKernelEx(&cfg, kern, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
