@@ -71,7 +71,7 @@ struct DecodeLayout {
     size_t blkidx = 0;        // int32 [batch, hkv, keep]       (hierarchical)
     size_t idx = 0;           // int32 [batch, hkv, B]
     size_t pm = 0, pl = 0, po = 0;
-    size_t counters = 0;      // uint64 [batch, hkv] attention split counters
+    size_t counters = 0;      // uint32 [batch, hkv] attention segment counters
     size_t hist = 0;          // uint32 [batch, hkv, 2048] order-key histogram (scorer -> top-B)
     size_t total = 0;
     lsa::AttnPlan plan{};
@@ -93,16 +93,16 @@ DecodeLayout decode_layout(const lsa_dims* d, int B, int blk, int keep, int num_
     L.idx = off;
     off = align_up(off + units * (size_t)B * 4);
     const int G = d->hq / d->hkv;
-    L.plan = lsa::plan_attn(d->batch, d->hkv, G, B, num_sms);
-    const size_t heads = (size_t)d->batch * d->hq;
+    L.plan = lsa::plan_attn(d->batch, d->hkv, G, B, d->d, num_sms);
+    const size_t slots = units * (size_t)L.plan.smax * G;
     L.pm = off;
-    off = align_up(off + heads * L.plan.nsw * 4);
+    off = align_up(off + slots * 4);
     L.pl = off;
-    off = align_up(off + heads * L.plan.nsw * 4);
+    off = align_up(off + slots * 4);
     L.po = off;
-    off = align_up(off + heads * L.plan.nsw * (size_t)d->d * 4);
+    off = align_up(off + slots * (size_t)d->d * 4);
     L.counters = off;
-    off = align_up(off + units * 8);
+    off = align_up(off + units * 4);
     L.hist = off;
     off = align_up(off + units * 2048 * 4);
     L.total = off;
@@ -187,7 +187,7 @@ lsa_status lsa_indexed_attn(const lsa_dims* dims, const lsa_bf16* q, const lsa_b
     if ((s = check_ws(ws, ws_bytes, L.total)) != LSA_OK) return s;
     return from_cuda(lsa::launch_attn(ctx, L.plan, q, k, v, idx, B, scale, out, at<float>(ws, L.pm),
                                       at<float>(ws, L.pl), at<float>(ws, L.po),
-                                      at<unsigned long long>(ws, L.counters), dims->batch, dims->hq, dims->hkv,
+                                      at<unsigned>(ws, L.counters), dims->batch, dims->hq, dims->hkv,
                                       dims->d, dims->T, (long long)dims->T * dims->hkv,
                                       at<unsigned>(ws, L.status)));
 }
@@ -249,7 +249,7 @@ lsa_status lsa_decode_step(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf
     }
     if (e == cudaSuccess)
         e = lsa::launch_attn(ctx, L.plan, q, k, v, idx, B, scale, out, at<float>(ws, L.pm), at<float>(ws, L.pl),
-                             at<float>(ws, L.po), at<unsigned long long>(ws, L.counters), dims->batch, dims->hq,
+                             at<float>(ws, L.po), at<unsigned>(ws, L.counters), dims->batch, dims->hq,
                              dims->hkv, dims->d, dims->T,
                              (long long)dims->T * dims->hkv, status);
     return from_cuda(e);

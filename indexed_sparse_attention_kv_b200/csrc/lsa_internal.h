@@ -54,9 +54,11 @@ struct LaunchCtx {
 };
 
 struct AttnPlan {
-    int rpc;      // index-set entries per CTA
-    int splits;   // CTAs per (row, KV head)
-    int nsw;      // partial slots per query head
+    long long units;          // rows x KV heads
+    int tiles_per_unit;       // ceil(B / 64)
+    long long total_tiles;
+    int ctas;                 // persistent CTAs (one wave)
+    int smax;                 // partial slots per unit
 };
 
 // mode 0: scores are the group-sum dot products (G x the mean); mode 1: means.
@@ -78,12 +80,13 @@ cudaError_t launch_centroids(const LaunchCtx& ctx, const uint16_t* kt, int blk, 
 cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int n, int B, int32_t* idx,
                         const int32_t* blkmap, int blk, int keep, uint32_t* ghist = nullptr);
 
-AttnPlan plan_attn(int nb, int hkv, int G, int B, int num_sms);
+AttnPlan plan_attn(int nb, int hkv, int G, int B, int d, int num_sms);
 
-// counters: [nb * hkv] zero-initialised; the kernel leaves them zero.
+// pm/pl: [units, smax, G] fp32, po: [units, smax, G, d] fp32, counters:
+// [units] uint32, zero on entry and left zero.
 cudaError_t launch_attn(const LaunchCtx& ctx, const AttnPlan& plan, const uint16_t* q, const uint16_t* k,
                         const uint16_t* v, const int32_t* idx, int B, float scale, uint16_t* out, float* pm, float* pl,
-                        float* po, unsigned long long* counters, int nb, int hq, int hkv, int d, int T,
+                        float* po, unsigned* counters, int nb, int hq, int hkv, int d, int T,
                         long long kv_bstride_rows, unsigned* status);
 
 }  // namespace lsa

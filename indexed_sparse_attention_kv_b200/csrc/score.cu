@@ -299,8 +299,10 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_launch_dependents();   // the selection kernel may start its prologue
     if (warp == kQConsumers) {
         if (lane == 0) {
+            const uint64_t stream_pol = policy_evict_first();   // read-once stream: keep it out of L2's way
             int issued = 0;
             for (int i = 0; i < nch; ++i) {
                 const int s = i % STAGES;
@@ -313,7 +315,7 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
                 const int ntok = min(tok, a.n - t0);
                 const uint32_t bytes = (uint32_t)(ntok * token_bytes);
                 mbar_arrive_expect_tx(&full[s], bytes);
-                bulk_g2s(stages + s * kQChunk, kt_b + (size_t)t0 * token_bytes, bytes, &full[s]);
+                bulk_g2s_hint(stages + s * kQChunk, kt_b + (size_t)t0 * token_bytes, bytes, &full[s], stream_pol);
                 issued = i + 1;
             }
             if (*abort_flag) {
@@ -339,6 +341,7 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
             for (int e = 0; e < 8; ++e) qv[k * 8 + e] = src[e];
         }
         float* out_h = a.out + ((size_t)b * hkv + head) * a.n;
+        const uint64_t keep_pol = policy_evict_last();   // the top-B selection re-reads the scores
         uint32_t* hs_h = hs + head * (kHistBins / 2);
         for (int i = 0; i < nch; ++i) {
             const int s = i % STAGES;
@@ -367,7 +370,7 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
                 acc += __shfl_xor_sync(0xffffffffu, acc, 1);
                 if (half == 0 && t < ntok) {
                     const float v = finalize_score(acc, a);
-                    out_h[t0 + t] = v;
+                    st_hint(out_h + t0 + t, v, keep_pol);
                     if (HIST) {
                         const uint32_t key = score_key(v);
                         if (key) atomicAdd(&hs_h[key >> 22], 1u << (((key >> 21) & 1u) * 16));

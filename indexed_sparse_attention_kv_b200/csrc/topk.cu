@@ -42,6 +42,7 @@ constexpr int kListPerWarp = 256;                       // (key, position) entri
 constexpr int kListCap = kListPerWarp * kTopkWarps;     // per CTA
 constexpr int kGatherCap = 4096;                        // bin-b0 keys of the whole cluster
 constexpr int kMaxCluster = 8;
+constexpr int kBatch = 8;                               // 128-key steps whose loads are issued together
 
 struct TopkArgs {
     const float* scores;      // [rows, n]
@@ -188,6 +189,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkAr
     const float* src = a.scores + (size_t)row * a.n + base;
     const bool vec = (a.n & 3) == 0;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_launch_dependents();
+    pdl_wait();   // the scores (and histogram) come from the previous kernel
     // warp sub-range of the segment, a multiple of 128 keys (4 per lane per step)
     int wlen = (len + kTopkWarps - 1) / kTopkWarps;
     wlen = (wlen + 127) & ~127;
@@ -200,12 +203,15 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkAr
     } else {
         for (int i = tid; i < kBins; i += kTopkThreads) sh.hist[i] = 0;
         __syncthreads();
-        for (int i0 = wbeg; i0 < wend; i0 += 128) {
-            uint32_t k[4];
-            load4(src, vec, i0 + lane * 4, wend, k);
+        for (int i00 = wbeg; i00 < wend; i00 += 128 * kBatch) {
+            uint32_t kk[kBatch][4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (k[u]) atomicAdd(&sh.hist[k[u] >> 21], 1u);
+            for (int ub = 0; ub < kBatch; ++ub) load4(src, vec, i00 + ub * 128 + lane * 4, wend, kk[ub]);
+#pragma unroll
+            for (int ub = 0; ub < kBatch; ++ub)
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (kk[ub][u]) atomicAdd(&sh.hist[kk[ub][u] >> 21], 1u);
         }
         cluster.sync();
         cluster_reduce(cluster, sh.hist, sh.red, kBins, CS);
@@ -222,30 +228,34 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkAr
     uint32_t* wkey = sh.lkey + warp * kListPerWarp;
     int* wpos = sh.lpos + warp * kListPerWarp;
     int wc = 0;
-    for (int i0 = wbeg; i0 < wend; i0 += 128) {
-        const int i = i0 + lane * 4;
-        uint32_t k[4];
-        load4(src, vec, i, wend, k);
-        bool f[4];
-        int c = 0;
+    for (int i00 = wbeg; i00 < wend; i00 += 128 * kBatch) {
+        uint32_t kk[kBatch][4];   // all loads of the batch in flight before any use
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            f[u] = k[u] != 0u && (k[u] >> 21) >= b0;
-            c += f[u];
-        }
-        int tot;
-        int slot = wc + warp_excl_scan(c, &tot);
+        for (int ub = 0; ub < kBatch; ++ub) load4(src, vec, i00 + ub * 128 + lane * 4, wend, kk[ub]);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (f[u]) {
-                if (slot < kListPerWarp) {
-                    wkey[slot] = k[u];
-                    wpos[slot] = base + i + u;
-                }
-                ++slot;
+        for (int ub = 0; ub < kBatch; ++ub) {
+            const int i = i00 + ub * 128 + lane * 4;
+            bool f[4];
+            int c = 0;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                f[u] = kk[ub][u] != 0u && (kk[ub][u] >> 21) >= b0;
+                c += f[u];
             }
+            int tot;
+            int slot = wc + warp_excl_scan(c, &tot);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (f[u]) {
+                    if (slot < kListPerWarp) {
+                        wkey[slot] = kk[ub][u];
+                        wpos[slot] = base + i + u;
+                    }
+                    ++slot;
+                }
+            }
+            wc += tot;
         }
-        wc += tot;
     }
     if (lane == 0) sh.wlist[warp] = wc;
     __syncthreads();
@@ -296,14 +306,26 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkAr
     const bool local_ok = !take_all && !any_over && ncand_all <= kGatherCap;
     (void)in_b0;
     if (local_ok) {
-        int off = 0;
+        // flattened gather: a thread's remote loads are independent, in flight together
+        int pre[kMaxCluster + 1];
+        pre[0] = 0;
 #pragma unroll
-        for (int rr = 0; rr < kMaxCluster; ++rr) {
-            if (rr < CS) {
-                const uint32_t* c = cluster.map_shared_rank(sh.cand, rr);
-                for (int i = tid; i < cnt[rr]; i += kTopkThreads) sh.gathered[off + i] = c[i];
-            }
-            off += cnt[rr];
+        for (int rr = 0; rr < kMaxCluster; ++rr) pre[rr + 1] = pre[rr] + cnt[rr];
+        const int off = pre[kMaxCluster];
+        constexpr int kG = kGatherCap / kTopkThreads;
+        uint32_t v[kG];
+#pragma unroll
+        for (int u = 0; u < kG; ++u) {
+            const int i = u * kTopkThreads + tid;
+            int rr = 0;
+#pragma unroll
+            for (int q = 1; q < kMaxCluster; ++q) rr += i >= pre[q];
+            v[u] = i < off ? cluster.map_shared_rank(sh.cand, rr)[i - pre[rr]] : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kG; ++u) {
+            const int i = u * kTopkThreads + tid;
+            if (i < off) sh.gathered[i] = v[u];
         }
         __syncthreads();
         uint32_t prefix = b0 << 21, pmask = 0xffe00000u;
@@ -500,13 +522,15 @@ cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int
     cfg.blockDim = dim3(kTopkThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = ctx.stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, kern, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
