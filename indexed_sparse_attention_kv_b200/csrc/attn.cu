@@ -8,16 +8,25 @@
 //
 // Work: unit u = (row b, KV head h) owns ceil(B / 64) tiles of 64 index-set
 // entries; the tiles of all units, in unit order, are cut into P contiguous
-// ranges, one per CTA (P = one wave: the SM count times the CTAs that fit).
-// A CTA streams its tiles through a kStages-deep ring: the selected K and V
-// rows and the unit's queries land in shared memory by 16-byte cp.async
-// (zero-fill for padded entries), the index rows of the tile kStages ahead are
-// read into registers one iteration early. Logits for the G heads are fp32 FMAs;
-// an online softmax in the exp2 domain accumulates (m, l, o) per query head over
-// the CTA's part of a unit (a segment). At a segment's end the CTA either
-// writes the output (the unit lies entirely in this CTA) or a partial; the last
-// CTA to finish a unit, found with a release/acquire counter, merges the unit's
-// partials and leaves the counter at zero.
+// ranges, one per CTA (P = one wave). A CTA streams its tiles through a
+// kStages-deep ring: the selected K and V rows land in shared memory by 16-byte
+// cp.async, 16 consecutive lanes per 256-byte row (coalesced), in an XOR
+// swizzle that keeps every ldmatrix phase conflict-free; padded entries are
+// zero-filled. The row ids of the tile kStages ahead are read one iteration
+// early. (Per-row TMA bulk copies were measured slower for 256-byte rows: the
+// copy engine, not DRAM, became the limit.)
+//
+// Compute (tensor cores, mma.sync m16n8k16, bf16 in, fp32 accumulate): the G
+// query heads are the M rows of one 16-row fragment (rows >= G are zero), and
+// warp w owns rows 16w .. 16w+15 of every tile, FlashAttention-2 style: it
+// forms its 16 logits per head, keeps a running max / sum per head in
+// registers, turns the probabilities (rounded to bf16, the operand type of the
+// instruction) straight from the logit fragments into the A operand of P.V,
+// and accumulates O[G x d] in registers. The 4 warps' states are merged through
+// shared memory at the end of a segment (the CTA's part of one unit). A unit
+// contained in one CTA is written directly; otherwise the CTA writes a partial
+// and the last one to finish a unit (a release/acquire counter, left at zero)
+// merges the unit's partials.
 #include <cuda_bf16.h>
 
 #include "lsa_common.cuh"
@@ -29,9 +38,7 @@ namespace {
 
 constexpr int kAttnThreads = 128;
 constexpr int kAttnWarps = 4;
-constexpr int kNT = 64;               // index-set entries per tile
-constexpr int kStages = 3;
-constexpr int kPS = kNT + 4;          // padded logit row (conflict-free fragment reads)
+constexpr int kNT = 64;               // index-set entries per tile (16 per warp)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttnArgs {
@@ -50,6 +57,7 @@ struct AttnArgs {
     long long total_tiles;
     float qscale;             // scale * log2(e)
     unsigned* status;
+    long long wait_limit;
 };
 
 // CTA that owns flattened tile w (ranges lo_p = p * W / P).
@@ -57,9 +65,8 @@ __device__ __forceinline__ int owner(long long w, const AttnArgs& a) {
     return (int)(((w + 1) * (long long)a.ctas - 1) / a.total_tiles);
 }
 
-// Swizzled position of 16-byte chunk c of tile row j: XOR with the row's low 3
-// bits, so that the 8 row addresses of every ldmatrix phase hit 8 distinct
-// 16-byte bank groups.
+// Swizzled position of 16-byte chunk c of tile row j: the 8 rows of an
+// ldmatrix phase hit 8 distinct 16-byte bank groups.
 __device__ __forceinline__ int swz(int j, int c) { return c ^ (j & 7); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
@@ -86,39 +93,39 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
+__device__ __forceinline__ float quad_max(float x) {
+    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
+    return fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
+}
+__device__ __forceinline__ float quad_sum(float x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    return x + __shfl_xor_sync(0xffffffffu, x, 2);
+}
 
 template <int D, int G>
 struct AttnLayout {
     static constexpr int kRowBytes = D * 2;
-    static constexpr int kKV = kNT * kRowBytes;                 // one of K or V per stage
-    static constexpr int kQ = G * D * 2;                         // the unit's queries (bf16)
-    static constexpr int kStage = 2 * kKV + kQ;                  // K, V, q
-    static constexpr int kP = G * (kNT + 4) * 4;                 // logits / weights (padded rows)
-    static constexpr int kHead = 3 * 16 * 4;                     // running max, sum, rescale per head
-    static constexpr int kRows = (kStages + 1) * kNT * 4;        // row-id ring
-    static constexpr int kTotal = kStages * kStage + kP + kHead + kRows;
+    static constexpr int kKV = kNT * kRowBytes;                    // one of K or V per stage
+    static constexpr int kQ = G * D * 2;                           // the unit's queries (bf16)
+    static constexpr int kStage = (2 * kKV + kQ + 127) / 128 * 128;
+    static constexpr int kMerge = (kAttnWarps - 1) * (G * D + 2 * 16) * 4;   // warps 1..3: O, m, l
+    static constexpr int kRows = 4 * kNT * 4;                      // row-id ring (>= stages + 1)
+    static constexpr int kFixed = kMerge + kRows;
+    static constexpr int kStages = (227 * 1024 / 2 - kFixed) / kStage >= 3 ? 3 : 2;
+    static constexpr int kTotal = kStages * kStage + kFixed;
 };
 
-// Tensor-core tile step (mma.sync m16n8k16, bf16 in, fp32 accumulate): the G
-// query heads are the M rows of one 16-row fragment (rows >= G are zero).
-//   logits  S[G x 64]  = Q[G x D] . K_tile^T   -- warp w: tile rows 16w .. 16w+15
-//   output  O[G x D]  += P[G x 64] . V_tile    -- warp w: dims w*D/4 .. (w+1)*D/4-1
-// P is rounded to bf16 for the product (the operand type of the tensor-core
-// instruction); m, l and the rescaling stay fp32.
 template <int D, int G>
 __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
     using Lay = AttnLayout<D, G>;
-    constexpr int CPR = D / 8;                 // 16-byte chunks per row
-    constexpr int QCH = G * D * 2 / 16;        // 16-byte chunks of the queries
+    constexpr int S = Lay::kStages;
     constexpr int KST = D / 16;                // k-steps of the logit product
-    constexpr int NTW = D / 32;                // 8-dim output tiles per warp
+    constexpr int NTO = D / 8;                 // 8-dim output tiles
+    static_assert(S + 1 <= 4, "row-id ring");
 
     extern __shared__ __align__(128) uint8_t smem[];
-    float* ps = reinterpret_cast<float*>(smem + kStages * Lay::kStage);
-    float* hm = ps + G * kPS;                  // running max per head (log2 domain)
-    float* hl = hm + 16;                       // running sum per head
-    float* ha = hl + 16;                       // rescale factor of the current tile
-    int* rowbuf = reinterpret_cast<int*>(ha + 16);
+    float* merge = reinterpret_cast<float*>(smem + S * Lay::kStage);
+    int* rowbuf = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(merge) + Lay::kMerge);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;    // mma fragment coordinates
@@ -145,20 +152,19 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
         }
         return t;
     };
-    // row ids of local tile i live in rowbuf[i % (kStages + 1)] from the
-    // iteration before it is issued until its compute is done
-    auto rows_of = [&](int i) { return rowbuf + (i % (kStages + 1)) * kNT; };
+    auto rows_of = [&](int i) { return rowbuf + (i & 3) * kNT; };
     // all threads issue local tile i: 16 consecutive lanes copy one 256-byte
     // row (coalesced), then the unit's queries; one commit group per call
     auto issue = [&](int i) {
         if (i < ntiles) {
-            uint8_t* st = smem + (i % kStages) * Lay::kStage;
+            uint8_t* st = smem + (i % S) * Lay::kStage;
             const int w = (int)(w0 + i);
             const int u = w / a.tiles_per_unit;
             const int b = u / a.hkv, h = u - b * a.hkv;
             const int* rows = rows_of(i);
             const uint8_t* kb = a.k + ((size_t)b * a.kv_bstride_rows + h) * Lay::kRowBytes;
             const uint8_t* vb = a.v + ((size_t)b * a.kv_bstride_rows + h) * Lay::kRowBytes;
+            constexpr int CPR = D / 8;
 #pragma unroll 4
             for (int id = tid; id < kNT * CPR; id += kAttnThreads) {
                 const int j = id / CPR, c = id - j * CPR;
@@ -170,185 +176,239 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
                 cp_async16(st + Lay::kKV + j * Lay::kRowBytes + pc * 16, vb + off, n);
             }
             const uint8_t* qs = reinterpret_cast<const uint8_t*>(a.q + ((size_t)b * a.hq + (size_t)h * G) * D);
-            for (int c = tid; c < QCH; c += kAttnThreads) cp_async16(st + 2 * Lay::kKV + c * 16, qs + c * 16, 16u);
+            for (int c = tid; c < Lay::kQ / 16; c += kAttnThreads) cp_async16(st + 2 * Lay::kKV + c * 16, qs + c * 16, 16u);
         }
         cp_async_commit();
     };
 
-    // prologue: ids of the first kStages tiles (loads issued together), then
-    // those tiles in flight, then the ids of the next tile in registers
+    // prologue: ids of the first S tiles (loads issued together), then those
+    // tiles in flight, then the ids of the next tile in registers
     {
-        int t0[kStages];
+        int t0[S];
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) t0[s] = tid < kNT ? fetch_row(s, tid) : -1;
+        for (int s = 0; s < S; ++s) t0[s] = tid < kNT ? fetch_row(s, tid) : -1;
         if (tid < kNT)
 #pragma unroll
-            for (int s = 0; s < kStages; ++s) rows_of(s)[tid] = t0[s];
-        if (tid < 16) {
-            hm[tid] = -INFINITY;
-            hl[tid] = 0.f;
-        }
-        __syncthreads();
+            for (int s = 0; s < S; ++s) rows_of(s)[tid] = t0[s];
+        __syncthreads();   // ids visible
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) issue(s);
+        for (int s = 0; s < S; ++s) issue(s);
     }
-    int t_next = tid < kNT ? fetch_row(kStages, tid) : -1;
+    int t_next = tid < kNT ? fetch_row(S, tid) : -1;
 
-    float acc[NTW][4];
-#pragma unroll
-    for (int j = 0; j < NTW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+    // per-warp running state: heads g (c0/c1 rows) and g + 8 (c2/c3 rows)
+    float acc[NTO][4];
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    uint32_t qf[KST][4];
+    int cur_u = -1;
     __shared__ int s_last;
+#pragma unroll
+    for (int j = 0; j < NTO; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
 
     for (int i = 0; i < ntiles; ++i) {
-        const int s = i % kStages;
-        if (tid < kNT) rows_of(i + kStages)[tid] = t_next;   // ids of the tile issued below
-        cp_async_wait<kStages - 1>();
-        __syncthreads();
+        const int s = i % S;
+        if (tid < kNT) rows_of(i + S)[tid] = t_next;   // ids of the tile issued below
+        cp_async_wait<S - 1>();
+        __syncthreads();   // tile i visible to every thread
         const uint8_t* ks = smem + s * Lay::kStage;
         const uint8_t* vs = ks + Lay::kKV;
-        const uint32_t* qw = reinterpret_cast<const uint32_t*>(ks + 2 * Lay::kKV);
         const int* rows = rows_of(i);
         const int w = (int)(w0 + i);
         const int u = w / a.tiles_per_unit;
-
-        // ---- logits for tile rows 16w .. 16w+15 (two 8-row n-tiles)
-        {
-            float sacc[2][4];
-#pragma unroll
-            for (int n = 0; n < 2; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
-            const int mi = lane >> 3, r8 = lane & 7;
-            const int krow = (warp * 2 + (mi >> 1)) * 8 + r8;
+        if (u != cur_u) {   // a new unit: its query fragments (A operand, rows >= G zero)
+            cur_u = u;
+            const uint32_t* qw = reinterpret_cast<const uint32_t*>(ks + 2 * Lay::kKV);
 #pragma unroll
             for (int kk = 0; kk < KST; ++kk) {
-                uint32_t af[4];
-                af[0] = g < G ? qw[(g * D + kk * 16 + 2 * t4) >> 1] : 0u;
-                af[1] = g + 8 < G ? qw[((g + 8) * D + kk * 16 + 2 * t4) >> 1] : 0u;
-                af[2] = g < G ? qw[(g * D + kk * 16 + 8 + 2 * t4) >> 1] : 0u;
-                af[3] = g + 8 < G ? qw[((g + 8) * D + kk * 16 + 8 + 2 * t4) >> 1] : 0u;
-                uint32_t bf[4];
-                ldsm_x4(bf, ks + krow * Lay::kRowBytes + swz(krow, kk * 2 + (mi & 1)) * 16);
-                mma_bf16(sacc[0], af, bf[0], bf[1]);
-                mma_bf16(sacc[1], af, bf[2], bf[3]);
+                qf[kk][0] = g < G ? qw[(g * D + kk * 16 + 2 * t4) >> 1] : 0u;
+                qf[kk][1] = g + 8 < G ? qw[((g + 8) * D + kk * 16 + 2 * t4) >> 1] : 0u;
+                qf[kk][2] = g < G ? qw[(g * D + kk * 16 + 8 + 2 * t4) >> 1] : 0u;
+                qf[kk][3] = g + 8 < G ? qw[((g + 8) * D + kk * 16 + 8 + 2 * t4) >> 1] : 0u;
             }
+        }
+
+        // ---- logits of this warp's 16 tile rows (two 8-row n-tiles)
+        float sc[2][4];
+#pragma unroll
+        for (int n = 0; n < 2; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+        {
+            const int mi = lane >> 3, r8 = lane & 7;
+            const int krow = warp * 16 + (mi >> 1) * 8 + r8;
+            const uint8_t* kp = ks + krow * Lay::kRowBytes;
+#pragma unroll
+            for (int kk = 0; kk < KST; ++kk) {
+                uint32_t bf[4];
+                ldsm_x4(bf, kp + swz(krow, kk * 2 + (mi & 1)) * 16);
+                mma_bf16(sc[0], qf[kk], bf[0], bf[1]);
+                mma_bf16(sc[1], qf[kk], bf[2], bf[3]);
+            }
+        }
+        // ---- online softmax per head row (the 4 lanes of a quad hold one row)
+        float pr[2][4];
+        {
+            float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
             for (int n = 0; n < 2; ++n) {
-                const int r0 = (warp * 2 + n) * 8 + 2 * t4;
+                const int r0 = warp * 16 + n * 8 + 2 * t4;
                 const bool v0 = rows[r0] >= 0, v1 = rows[r0 + 1] >= 0;
-                if (g < G) {
-                    ps[g * kPS + r0] = v0 ? sacc[n][0] * a.qscale : -INFINITY;
-                    ps[g * kPS + r0 + 1] = v1 ? sacc[n][1] * a.qscale : -INFINITY;
-                }
-                if (g + 8 < G) {
-                    ps[(g + 8) * kPS + r0] = v0 ? sacc[n][2] * a.qscale : -INFINITY;
-                    ps[(g + 8) * kPS + r0 + 1] = v1 ? sacc[n][3] * a.qscale : -INFINITY;
-                }
+                sc[n][0] = v0 ? sc[n][0] * a.qscale : -INFINITY;
+                sc[n][1] = v1 ? sc[n][1] * a.qscale : -INFINITY;
+                sc[n][2] = v0 ? sc[n][2] * a.qscale : -INFINITY;
+                sc[n][3] = v1 ? sc[n][3] * a.qscale : -INFINITY;
+                mx0 = fmaxf(mx0, fmaxf(sc[n][0], sc[n][1]));
+                mx1 = fmaxf(mx1, fmaxf(sc[n][2], sc[n][3]));
             }
-        }
-        __syncthreads();
-
-        // ---- online softmax per head (warp w: heads w, w + 4, ...)
-        for (int hh = warp; hh < G; hh += kAttnWarps) {
-            float* pg = ps + hh * kPS;
-            const float x0 = pg[lane], x1 = pg[lane + 32];
-            const float tmax = warp_max(fmaxf(x0, x1));
-            const float m_old = hm[hh];
-            const float m_new = fmaxf(m_old, tmax);
-            float e0 = 0.f, e1 = 0.f, alpha = 1.f;
-            if (m_new != -INFINITY) {
-                alpha = exp2f(m_old - m_new);
-                e0 = exp2f(x0 - m_new);
-                e1 = exp2f(x1 - m_new);
-            }
-            pg[lane] = e0;
-            pg[lane + 32] = e1;
-            const float lsum = warp_sum(e0 + e1);
-            if (lane == 0) {
-                hl[hh] = hl[hh] * alpha + lsum;
-                hm[hh] = m_new;
-                ha[hh] = alpha;
-            }
-        }
-        __syncthreads();
-
-        // ---- rescale and accumulate P . V for this warp's dims
-        {
-            const float al0 = g < G ? ha[g] : 1.f, al1 = g + 8 < G ? ha[g + 8] : 1.f;
+            mx0 = quad_max(mx0);
+            mx1 = quad_max(mx1);
+            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+            const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m0 - mn0);
+            const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m1 - mn1);
+            float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < NTW; ++j) {
+            for (int n = 0; n < 2; ++n) {
+                pr[n][0] = mn0 == -INFINITY ? 0.f : exp2f(sc[n][0] - mn0);
+                pr[n][1] = mn0 == -INFINITY ? 0.f : exp2f(sc[n][1] - mn0);
+                pr[n][2] = mn1 == -INFINITY ? 0.f : exp2f(sc[n][2] - mn1);
+                pr[n][3] = mn1 == -INFINITY ? 0.f : exp2f(sc[n][3] - mn1);
+                s0 += pr[n][0] + pr[n][1];
+                s1 += pr[n][2] + pr[n][3];
+            }
+            l0 = l0 * al0 + quad_sum(s0);
+            l1 = l1 * al1 + quad_sum(s1);
+            m0 = mn0;
+            m1 = mn1;
+#pragma unroll
+            for (int j = 0; j < NTO; ++j) {
                 acc[j][0] *= al0;
                 acc[j][1] *= al0;
                 acc[j][2] *= al1;
                 acc[j][3] *= al1;
             }
+        }
+        // ---- O += P . V over this warp's 16 rows (one k-step)
+        {
+            uint32_t af[4];
+            af[0] = pack_bf16(pr[0][0], pr[0][1]);
+            af[1] = pack_bf16(pr[0][2], pr[0][3]);
+            af[2] = pack_bf16(pr[1][0], pr[1][1]);
+            af[3] = pack_bf16(pr[1][2], pr[1][3]);
             const int mi = lane >> 3, r8 = lane & 7;
+            const int vrow = warp * 16 + (mi & 1) * 8 + r8;
+            const uint8_t* vp = vs + vrow * Lay::kRowBytes;
 #pragma unroll
-            for (int kq = 0; kq < kNT / 16; ++kq) {
-                uint32_t af[4];
-                const int c0 = kq * 16 + 2 * t4;
-                af[0] = g < G ? pack_bf16(ps[g * kPS + c0], ps[g * kPS + c0 + 1]) : 0u;
-                af[1] = g + 8 < G ? pack_bf16(ps[(g + 8) * kPS + c0], ps[(g + 8) * kPS + c0 + 1]) : 0u;
-                af[2] = g < G ? pack_bf16(ps[g * kPS + c0 + 8], ps[g * kPS + c0 + 9]) : 0u;
-                af[3] = g + 8 < G ? pack_bf16(ps[(g + 8) * kPS + c0 + 8], ps[(g + 8) * kPS + c0 + 9]) : 0u;
-                const int vrow = kq * 16 + (mi & 1) * 8 + r8;
-#pragma unroll
-                for (int j = 0; j < NTW; j += 2) {
-                    const int nt = warp * NTW + j + (mi >> 1);
-                    uint32_t bf[4];
-                    ldsm_x4_t(bf, vs + vrow * Lay::kRowBytes + swz(vrow, nt) * 16);
-                    mma_bf16(acc[j], af, bf[0], bf[1]);
-                    mma_bf16(acc[j + 1], af, bf[2], bf[3]);
-                }
+            for (int j = 0; j < NTO; j += 2) {
+                uint32_t bf[4];
+                ldsm_x4_t(bf, vp + swz(vrow, j + (mi >> 1)) * 16);
+                mma_bf16(acc[j], af, bf[0], bf[1]);
+                mma_bf16(acc[j + 1], af, bf[2], bf[3]);
             }
         }
-        __syncthreads();   // stage s and the logits are free again
 
-        // refill stage s with tile i + kStages; fetch the ids one tile further
-        issue(i + kStages);
-        t_next = tid < kNT ? fetch_row(i + kStages + 1, tid) : -1;
+        __syncthreads();   // stage s free once every warp is done with it
+        issue(i + S);
+        t_next = tid < kNT ? fetch_row(i + S + 1, tid) : -1;
 
         // ---- end of a segment: this CTA's last tile of unit u
         const bool seg_end = i + 1 == ntiles || (w + 1) / a.tiles_per_unit != u;
         if (!seg_end) continue;
+        // merge the 4 warps' states into warp 0 (rows g and g + 8 of each)
+        if (warp > 0) {
+            float* mw = merge + (warp - 1) * (G * D + 32);
+            if (t4 == 0) {
+                mw[G * D + g] = m0;
+                mw[G * D + 16 + g] = l0;
+                if (g + 8 < 16) {
+                    mw[G * D + g + 8] = m1;
+                    mw[G * D + 16 + g + 8] = l1;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < NTO; ++j) {
+                const int d0 = j * 8 + 2 * t4;
+                if (g < G) *reinterpret_cast<float2*>(mw + g * D + d0) = make_float2(acc[j][0], acc[j][1]);
+                if (g + 8 < G) *reinterpret_cast<float2*>(mw + (g + 8) * D + d0) = make_float2(acc[j][2], acc[j][3]);
+            }
+        }
+        __syncthreads();
         const int b = u / a.hkv, h = u - b * a.hkv;
         const long long wu0 = (long long)u * a.tiles_per_unit;
         const int pfirst = owner(wu0, a);
         const int nslot = owner(wu0 + a.tiles_per_unit - 1, a) - pfirst + 1;
-        if (nslot == 1) {
-            // the whole unit lies in this CTA: write the output directly
+        if (warp == 0) {
+            float M0 = m0, M1 = m1;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int hd = g + 8 * half;
-                if (hd < G) {
-                    const float l = hl[hd];
-                    const float inv = l > 0.f ? 1.f / l : 0.f;
-                    uint16_t* o = a.out + ((size_t)b * a.hq + h * G + hd) * D;
+            for (int x = 0; x < kAttnWarps - 1; ++x) {
+                const float* mw = merge + x * (G * D + 32);
+                M0 = fmaxf(M0, mw[G * D + g]);
+                M1 = fmaxf(M1, g + 8 < 16 ? mw[G * D + g + 8] : -INFINITY);
+            }
+            float w00 = M0 == -INFINITY ? 0.f : exp2f(m0 - M0), w10 = M1 == -INFINITY ? 0.f : exp2f(m1 - M1);
+            float L0 = w00 * l0, L1 = w10 * l1;
 #pragma unroll
-                    for (int j = 0; j < NTW; ++j) {
-                        const int d0 = (warp * NTW + j) * 8 + 2 * t4;
-                        *reinterpret_cast<uint32_t*>(o + d0) =
-                            pack_bf16(acc[j][2 * half] * inv, acc[j][2 * half + 1] * inv);
+            for (int j = 0; j < NTO; ++j) {
+                acc[j][0] *= w00;
+                acc[j][1] *= w00;
+                acc[j][2] *= w10;
+                acc[j][3] *= w10;
+            }
+#pragma unroll
+            for (int x = 0; x < kAttnWarps - 1; ++x) {
+                const float* mw = merge + x * (G * D + 32);
+                const float wx0 = M0 == -INFINITY ? 0.f : exp2f(mw[G * D + g] - M0);
+                const float wx1 = M1 == -INFINITY ? 0.f : exp2f(mw[G * D + g + 8] - M1);
+                L0 = fmaf(wx0, mw[G * D + 16 + g], L0);
+                L1 = fmaf(wx1, mw[G * D + 16 + g + 8], L1);
+#pragma unroll
+                for (int j = 0; j < NTO; ++j) {
+                    const int d0 = j * 8 + 2 * t4;
+                    if (g < G) {
+                        const float2 o = *reinterpret_cast<const float2*>(mw + g * D + d0);
+                        acc[j][0] = fmaf(wx0, o.x, acc[j][0]);
+                        acc[j][1] = fmaf(wx0, o.y, acc[j][1]);
+                    }
+                    if (g + 8 < G) {
+                        const float2 o = *reinterpret_cast<const float2*>(mw + (g + 8) * D + d0);
+                        acc[j][2] = fmaf(wx1, o.x, acc[j][2]);
+                        acc[j][3] = fmaf(wx1, o.y, acc[j][3]);
                     }
                 }
             }
-        } else {
-            const int slot = p - pfirst;
+            if (nslot == 1) {
+                // the whole unit lies in this CTA: write the output directly
+                const float i0 = L0 > 0.f ? 1.f / L0 : 0.f, i1 = L1 > 0.f ? 1.f / L1 : 0.f;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int hd = g + 8 * half;
-                if (hd < G) {
-                    const size_t pi = ((size_t)u * a.smax + slot) * G + hd;
-                    if (warp == 0 && t4 == 0) {
-                        a.pm[pi] = hm[hd];
-                        a.pl[pi] = hl[hd];
+                for (int j = 0; j < NTO; ++j) {
+                    const int d0 = j * 8 + 2 * t4;
+                    if (g < G)
+                        *reinterpret_cast<uint32_t*>(a.out + ((size_t)b * a.hq + h * G + g) * D + d0) =
+                            pack_bf16(acc[j][0] * i0, acc[j][1] * i0);
+                    if (g + 8 < G)
+                        *reinterpret_cast<uint32_t*>(a.out + ((size_t)b * a.hq + h * G + g + 8) * D + d0) =
+                            pack_bf16(acc[j][2] * i1, acc[j][3] * i1);
+                }
+            } else {
+                const int slot = p - pfirst;
+                const size_t pi0 = ((size_t)u * a.smax + slot) * G + g;
+                if (t4 == 0) {
+                    if (g < G) {
+                        a.pm[pi0] = M0;
+                        a.pl[pi0] = L0;
                     }
-                    float* po = a.po + pi * D;
-#pragma unroll
-                    for (int j = 0; j < NTW; ++j) {
-                        const int d0 = (warp * NTW + j) * 8 + 2 * t4;
-                        *reinterpret_cast<float2*>(po + d0) = make_float2(acc[j][2 * half], acc[j][2 * half + 1]);
+                    if (g + 8 < G) {
+                        a.pm[pi0 + 8] = M1;
+                        a.pl[pi0 + 8] = L1;
                     }
                 }
+#pragma unroll
+                for (int j = 0; j < NTO; ++j) {
+                    const int d0 = j * 8 + 2 * t4;
+                    if (g < G) *reinterpret_cast<float2*>(a.po + pi0 * D + d0) = make_float2(acc[j][0], acc[j][1]);
+                    if (g + 8 < G)
+                        *reinterpret_cast<float2*>(a.po + (pi0 + 8) * D + d0) = make_float2(acc[j][2], acc[j][3]);
+                }
             }
+        }
+        if (nslot > 1) {
             __syncthreads();
             if (tid == 0) {
                 unsigned old;
@@ -359,8 +419,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
             __syncthreads();
             if (s_last) {
                 __threadfence();
-                // merge the unit's nslot partials: warp -> heads, lanes -> slots for
-                // the weights, then lanes -> dims with every slot's loads in flight
+                // merge the unit's nslot partials: warp -> heads; lanes -> slots for
+                // the weights, then lanes -> dims with 16 slots' loads in flight
                 constexpr int DPL = D / 32;
                 for (int hd = warp; hd < G; hd += kAttnWarps) {
                     const size_t base = (size_t)u * a.smax * G + hd;
@@ -371,24 +431,29 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
 #pragma unroll
                     for (int k = 0; k < DPL; ++k) oacc[k] = 0.f;
                     if (M != -INFINITY) {
-                        for (int x0 = 0; x0 < nslot; x0 += 8) {
-                            float wv[8], vals[8][DPL];
+                        for (int x0 = 0; x0 < nslot; x0 += 32) {
+                            const int xl = x0 + lane;
+                            const float mx = xl < nslot ? __ldcg(a.pm + base + (size_t)xl * G) : -INFINITY;
+                            const float lx = xl < nslot ? __ldcg(a.pl + base + (size_t)xl * G) : 0.f;
+                            const float wl = mx == -INFINITY ? 0.f : exp2f(mx - M);
+                            L += warp_sum(wl * lx);
+                            const int cnt = min(32, nslot - x0);
+                            for (int y0 = 0; y0 < cnt; y0 += 16) {
+                                float vals[16][DPL];
 #pragma unroll
-                            for (int y = 0; y < 8; ++y) {
-                                const int x = x0 + y;
-                                const size_t pi = base + (size_t)x * G;
-                                const float mx = x < nslot ? __ldcg(a.pm + pi) : -INFINITY;
-                                wv[y] = mx == -INFINITY ? 0.f : exp2f(mx - M);
-                                const float lx = x < nslot ? __ldcg(a.pl + pi) : 0.f;
-                                L = fmaf(wv[y], lx, L);
+                                for (int y = 0; y < 16; ++y)
 #pragma unroll
-                                for (int k = 0; k < DPL; ++k)
-                                    vals[y][k] = x < nslot ? __ldcg(a.po + pi * D + lane * DPL + k) : 0.f;
+                                    for (int k = 0; k < DPL; ++k)
+                                        vals[y][k] = y0 + y < cnt
+                                                         ? __ldcg(a.po + (base + (size_t)(x0 + y0 + y) * G) * D + lane * DPL + k)
+                                                         : 0.f;
+#pragma unroll
+                                for (int y = 0; y < 16; ++y) {
+                                    const float wy = __shfl_sync(0xffffffffu, wl, (y0 + y) & 31);
+#pragma unroll
+                                    for (int k = 0; k < DPL; ++k) oacc[k] = fmaf(wy, vals[y][k], oacc[k]);
+                                }
                             }
-#pragma unroll
-                            for (int y = 0; y < 8; ++y)
-#pragma unroll
-                                for (int k = 0; k < DPL; ++k) oacc[k] = fmaf(wv[y], vals[y][k], oacc[k]);
                         }
                     }
                     const float inv = L > 0.f ? 1.f / L : 0.f;
@@ -398,15 +463,13 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
                 }
             }
         }
-        // next segment: fresh state (the barrier at the top of the next
-        // iteration orders these resets before their first use)
+        // next segment: fresh state (the merge buffer is reused only after the
+        // next segment end's barrier)
 #pragma unroll
-        for (int j = 0; j < NTW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+        for (int j = 0; j < NTO; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
         __syncthreads();
-        if (tid < 16) {
-            hm[tid] = -INFINITY;
-            hl[tid] = 0.f;
-        }
     }
     cp_async_wait<0>();
 }
@@ -464,7 +527,7 @@ AttnPlan plan_attn(int nb, int hkv, int G, int B, int d, int num_sms) {
     p.tiles_per_unit = (B + kNT - 1) / kNT;
     p.total_tiles = p.units * p.tiles_per_unit;
     const size_t smem = d == 64 ? smem_d<64>(G) : (d == 128 ? smem_d<128>(G) : smem_d<256>(G));
-    int per_sm = (int)(227 * 1024 / (smem + 1024));
+    int per_sm = (int)(228 * 1024 / (smem + 1024));
     if (per_sm > 4) per_sm = 4;
     if (per_sm < 1) per_sm = 1;
     long long ctas = (long long)num_sms * per_sm;
@@ -503,6 +566,7 @@ cudaError_t launch_attn(const LaunchCtx& ctx, const AttnPlan& plan, const uint16
     a.total_tiles = plan.total_tiles;
     a.qscale = scale * kLog2e;
     a.status = status;
+    a.wait_limit = ctx.wait_limit;
     (void)nb;
     const int G = hq / hkv;
     switch (d) {

@@ -15,12 +15,13 @@
 //   2. One pass over the keys in position order: every warp appends the
 //      (key, position) pairs of bin >= b0 to its own list (about B plus the
 //      threshold bin's keys per row: a small fraction of the row).
-//   3. The keys of bin b0 of the whole cluster are gathered in every CTA and two
-//      local radix passes give the exact threshold key theta and the number of
-//      ties at theta to take.
-//   4. Counts above / at theta per warp, exclusive prefix sums over warps and
-//      over the cluster's CTAs, and a ballot compaction of the short lists write
-//      the positions in ascending order.
+//   3. The keys of bin b0 of the whole cluster (in rank, hence position,
+//      order) are gathered in every CTA; two local radix passes give the exact
+//      threshold key theta and the number of ties at theta to take, and from
+//      the same keys and the per-CTA list lengths every CTA derives its tie
+//      quota and output offset: no further exchange.
+//   4. Counts above / at theta per warp and a ballot compaction of the short
+//      lists write the positions in ascending order.
 // Whenever a list or the threshold bin is too large for shared memory (e.g.
 // many equal scores), the cluster switches, uniformly, to radix passes and a
 // compaction over the keys themselves, with the same result.
@@ -38,7 +39,7 @@ namespace {
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kBins = 2048;
-constexpr int kListPerWarp = 256;                       // (key, position) entries per warp
+constexpr int kListPerWarp = 128;                       // (key, position) entries per warp
 constexpr int kListCap = kListPerWarp * kTopkWarps;     // per CTA
 constexpr int kGatherCap = 4096;                        // bin-b0 keys of the whole cluster
 constexpr int kMaxCluster = 8;
@@ -57,46 +58,18 @@ struct TopkShared {
     uint32_t hist[kBins];           // this CTA's histogram / local refinement histogram
     uint32_t lkey[kListCap];        // per-warp lists (position order) of keys in bins >= b0
     int lpos[kListCap];
-    uint32_t cand[kListCap];        // this CTA's bin-b0 keys (any order)
+    uint32_t cand[kListCap];        // this CTA's bin-b0 keys (position order)
     uint32_t gathered[kGatherCap];  // the cluster's bin-b0 keys
     int wlist[kTopkWarps], wb0[kTopkWarps];
     int scan[kTopkWarps];
     int warp_gt[kTopkWarps], warp_eq[kTopkWarps];
     int warp_sel_before[kTopkWarps], warp_eq_before[kTopkWarps];
-    int cta_gt, cta_eq, ncand, overflow;
+    int cta_gt, cta_eq, ncand, nlist, overflow;
+    int rcnt[2 * kMaxCluster];      // per rank: gathered keys above / at theta
     uint32_t bstar;
     int above;
     int total;
 };
-
-// Exclusive prefix sum over the CTA's threads (thread order); returns the
-// exclusive prefix, and the CTA total through *total.
-__device__ __forceinline__ int block_excl_scan(int v, int* scan, int* total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) scan[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < kTopkWarps ? scan[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += y;
-        }
-        if (lane < kTopkWarps) scan[lane] = w;   // inclusive per warp
-    }
-    __syncthreads();
-    const int warp_excl = warp ? scan[warp - 1] : 0;
-    const int res = warp_excl + x - v;
-    *total = scan[kTopkWarps - 1];
-    __syncthreads();
-    return res;
-}
 
 // Warp-level exclusive prefix sum; *total = the warp's sum.
 __device__ __forceinline__ int warp_excl_scan(int v, int* total) {
@@ -117,10 +90,27 @@ __device__ __forceinline__ int warp_excl_scan(int v, int* total) {
 __device__ __forceinline__ int find_bin(const uint32_t* red, int nb, int krem, TopkShared& sh) {
     const int per = nb / kTopkThreads;
     const int hi = nb - 1 - (int)threadIdx.x * per;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int local = 0;
     for (int q = 0; q < per; ++q) local += (int)red[hi - q];
-    int total;
-    const int above_me = block_excl_scan(local, sh.scan, &total);
+    // two barriers: warp scans, warp totals through shared memory, then every
+    // thread adds the totals of the warps above it
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) sh.scan[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kTopkWarps; ++w) {
+        const int t = sh.scan[w];
+        before += w < warp ? t : 0;
+        total += t;
+    }
+    const int above_me = before + incl - local;
     if (above_me < krem && krem <= above_me + local) {
         int cum = above_me;
         for (int q = 0; q < per; ++q) {
@@ -174,8 +164,31 @@ __device__ __forceinline__ void load4(const float* src, bool vec, int i, int end
     }
 }
 
+// kBatch 128-key steps of a warp range starting at i00 (lane: 4 consecutive
+// keys per step): every load is issued before any key is converted, so a
+// thread's loads are all in flight together.
+__device__ __forceinline__ void load_batch(const float* src, bool vec, int i00, int end, int lane,
+                                           uint32_t (&kk)[kBatch][4]) {
+    if (vec && i00 + 128 * kBatch <= end) {
+        float4 v[kBatch];
+#pragma unroll
+        for (int ub = 0; ub < kBatch; ++ub)
+            v[ub] = __ldcg(reinterpret_cast<const float4*>(src + i00 + ub * 128 + lane * 4));
+#pragma unroll
+        for (int ub = 0; ub < kBatch; ++ub) {
+            kk[ub][0] = score_key(v[ub].x);
+            kk[ub][1] = score_key(v[ub].y);
+            kk[ub][2] = score_key(v[ub].z);
+            kk[ub][3] = score_key(v[ub].w);
+        }
+    } else {
+#pragma unroll
+        for (int ub = 0; ub < kBatch; ++ub) load4(src, vec, i00 + ub * 128 + lane * 4, end, kk[ub]);
+    }
+}
+
 template <bool EXT_HIST>
-__global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkArgs a) {
+__global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster_kernel(const TopkArgs a) {
     cg::cluster_group cluster = cg::this_cluster();
     const int CS = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
@@ -205,8 +218,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkAr
         __syncthreads();
         for (int i00 = wbeg; i00 < wend; i00 += 128 * kBatch) {
             uint32_t kk[kBatch][4];
-#pragma unroll
-            for (int ub = 0; ub < kBatch; ++ub) load4(src, vec, i00 + ub * 128 + lane * 4, wend, kk[ub]);
+            load_batch(src, vec, i00, wend, lane, kk);
 #pragma unroll
             for (int ub = 0; ub < kBatch; ++ub)
 #pragma unroll
@@ -225,36 +237,33 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkAr
     const int in_b0 = take_all ? 0 : (int)sh.red[b0];
 
     // ---- 2. per-warp lists of (key, position) with bin >= b0, in position order
+    // Coalesced steps of 128 keys (lane: 4 consecutive keys, one 16-byte load;
+    // every load of a batch issued before any use); four ballots per step give
+    // each hit its rank in position order without a shuffle scan.
     uint32_t* wkey = sh.lkey + warp * kListPerWarp;
     int* wpos = sh.lpos + warp * kListPerWarp;
     int wc = 0;
+    const unsigned lt = (1u << lane) - 1u;
     for (int i00 = wbeg; i00 < wend; i00 += 128 * kBatch) {
-        uint32_t kk[kBatch][4];   // all loads of the batch in flight before any use
-#pragma unroll
-        for (int ub = 0; ub < kBatch; ++ub) load4(src, vec, i00 + ub * 128 + lane * 4, wend, kk[ub]);
+        uint32_t kk[kBatch][4];
+        load_batch(src, vec, i00, wend, lane, kk);
 #pragma unroll
         for (int ub = 0; ub < kBatch; ++ub) {
-            const int i = i00 + ub * 128 + lane * 4;
-            bool f[4];
-            int c = 0;
+            unsigned m[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) m[u] = __ballot_sync(0xffffffffu, kk[ub][u] != 0u && (kk[ub][u] >> 21) >= b0);
+            int slot = wc + __popc(m[0] & lt) + __popc(m[1] & lt) + __popc(m[2] & lt) + __popc(m[3] & lt);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                f[u] = kk[ub][u] != 0u && (kk[ub][u] >> 21) >= b0;
-                c += f[u];
-            }
-            int tot;
-            int slot = wc + warp_excl_scan(c, &tot);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (f[u]) {
+                if ((m[u] >> lane) & 1u) {
                     if (slot < kListPerWarp) {
                         wkey[slot] = kk[ub][u];
-                        wpos[slot] = base + i + u;
+                        wpos[slot] = base + i00 + ub * 128 + lane * 4 + u;
                     }
                     ++slot;
                 }
             }
-            wc += tot;
+            wc += __popc(m[0]) + __popc(m[1]) + __popc(m[2]) + __popc(m[3]);
         }
     }
     if (lane == 0) sh.wlist[warp] = wc;
@@ -262,7 +271,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkAr
     bool over = false;
     for (int w = 0; w < kTopkWarps; ++w) over |= sh.wlist[w] > kListPerWarp;
     if (!take_all && !over) {
-        // pack this CTA's bin-b0 keys for the cluster gather
+        // pack this CTA's bin-b0 keys (position order) for the cluster gather
         int nb0 = 0;
         for (int j = lane; j < ((wc + 31) & ~31); j += 32) {
             const bool hit = j < wc && (wkey[j] >> 21) == b0;
@@ -279,183 +288,42 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkAr
             if (hit) sh.cand[off + __popc(m & ((1u << lane) - 1u))] = wkey[j];
             off += __popc(m);
         }
-        if (tid == 0) {
-            int t = 0;
-            for (int w = 0; w < kTopkWarps; ++w) t += sh.wb0[w];
-            sh.ncand = t;
-        }
     }
-    if (tid == 0) sh.overflow = over;
-    cluster.sync();   // lists, packed keys and flags complete; every CTA has read the row histogram
+    if (tid == 0) {
+        int nl = 0, nc = 0;
+        for (int w = 0; w < kTopkWarps; ++w) {
+            nl += sh.wlist[w];
+            nc += (!take_all && !over) ? sh.wb0[w] : 0;
+        }
+        sh.nlist = nl;
+        sh.ncand = nc;
+        sh.overflow = over;
+    }
+    cluster.sync();   // lists, packed keys and counts complete; every CTA has read the row histogram
     if (EXT_HIST && rank == 0)
         for (int i = tid; i < kBins; i += kTopkThreads) a.ghist[(size_t)row * kBins + i] = 0u;
-    int any_over = 0;
-#pragma unroll
-    for (int rr = 0; rr < kMaxCluster; ++rr) any_over |= rr < CS ? cluster.map_shared_rank(&sh, rr)->overflow : 0;
-
-    // ---- 3. exact threshold theta and the ties at theta to take
-    uint32_t theta = 0;
-    int cnt[kMaxCluster];
-    int ncand_all = 0;
+    int any_over = 0, cnt[kMaxCluster], nl[kMaxCluster];
 #pragma unroll
     for (int rr = 0; rr < kMaxCluster; ++rr) {
-        cnt[rr] = (rr < CS && !take_all && !any_over) ? cluster.map_shared_rank(&sh, rr)->ncand : 0;
-        ncand_all += cnt[rr];
+        const TopkShared* o = cluster.map_shared_rank(&sh, rr < CS ? rr : 0);
+        any_over |= rr < CS ? o->overflow : 0;
+        cnt[rr] = rr < CS ? o->ncand : 0;
+        nl[rr] = rr < CS ? o->nlist : 0;
     }
-    // the packed counts, not the histogram, decide: the gather can never overrun
-    const bool local_ok = !take_all && !any_over && ncand_all <= kGatherCap;
+    int pre[kMaxCluster + 1];
+    pre[0] = 0;
+#pragma unroll
+    for (int rr = 0; rr < kMaxCluster; ++rr) pre[rr + 1] = pre[rr] + cnt[rr];
+    const int ncand_all = pre[kMaxCluster];
     (void)in_b0;
-    if (local_ok) {
-        // flattened gather: a thread's remote loads are independent, in flight together
-        int pre[kMaxCluster + 1];
-        pre[0] = 0;
-#pragma unroll
-        for (int rr = 0; rr < kMaxCluster; ++rr) pre[rr + 1] = pre[rr] + cnt[rr];
-        const int off = pre[kMaxCluster];
-        constexpr int kG = kGatherCap / kTopkThreads;
-        uint32_t v[kG];
-#pragma unroll
-        for (int u = 0; u < kG; ++u) {
-            const int i = u * kTopkThreads + tid;
-            int rr = 0;
-#pragma unroll
-            for (int q = 1; q < kMaxCluster; ++q) rr += i >= pre[q];
-            v[u] = i < off ? cluster.map_shared_rank(sh.cand, rr)[i - pre[rr]] : 0u;
-        }
-#pragma unroll
-        for (int u = 0; u < kG; ++u) {
-            const int i = u * kTopkThreads + tid;
-            if (i < off) sh.gathered[i] = v[u];
-        }
-        __syncthreads();
-        uint32_t prefix = b0 << 21, pmask = 0xffe00000u;
-        for (int pass = 1; pass < 3; ++pass) {
-            const int shift = pass == 1 ? 10 : 0;
-            const int nb = pass == 1 ? 2048 : 1024;
-            for (int i = tid; i < nb; i += kTopkThreads) sh.hist[i] = 0;
-            __syncthreads();
-            for (int i = tid; i < off; i += kTopkThreads) {
-                const uint32_t k = sh.gathered[i];
-                if ((k & pmask) == prefix) atomicAdd(&sh.hist[(k >> shift) & (uint32_t)(nb - 1)], 1u);
-            }
-            __syncthreads();
-            find_bin(sh.hist, nb, krem, sh);
-            prefix |= sh.bstar << shift;
-            pmask |= (uint32_t)(nb - 1) << shift;
-            krem -= sh.above;
-            __syncthreads();
-        }
-        theta = prefix;
-    }
-    cluster.sync();   // remote reads of the packed keys are done
-    if (!take_all && !local_ok) {
-        // too many keys for shared memory: resolve the low 21 bits with
-        // cluster-wide radix passes over the keys themselves
-        uint32_t prefix = b0 << 21, pmask = 0xffe00000u;
-        for (int pass = 1; pass < 3; ++pass) {
-            const int shift = pass == 1 ? 10 : 0;
-            const int nb = pass == 1 ? 2048 : 1024;
-            for (int i = tid; i < nb; i += kTopkThreads) sh.hist[i] = 0;
-            __syncthreads();
-            for (int i0 = wbeg; i0 < wend; i0 += 128) {
-                uint32_t k[4];
-                load4(src, vec, i0 + lane * 4, wend, k);
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    if (k[u] && (k[u] & pmask) == prefix) atomicAdd(&sh.hist[(k[u] >> shift) & (uint32_t)(nb - 1)], 1u);
-            }
-            cluster.sync();
-            cluster_reduce(cluster, sh.hist, sh.red, nb, CS);
-            cluster.sync();   // hist may be reset next pass only after every CTA has read it
-            find_bin(sh.red, nb, krem, sh);
-            prefix |= sh.bstar << shift;
-            pmask |= (uint32_t)(nb - 1) << shift;
-            krem -= sh.above;
-            __syncthreads();
-        }
-        theta = prefix;
-    }
-    if (take_all) krem = 0;   // every valid key (key > 0 = theta) is taken
-
-    // ---- 4. counts per warp (position order), offsets, compaction
-    int gt = 0, eq = 0;
-    if (!any_over) {
-        for (int j = lane; j < wc; j += 32) {
-            const uint32_t k = wkey[j];
-            gt += k > theta;
-            eq += k == theta;
-        }
-    } else {
-        for (int i0 = wbeg; i0 < wend; i0 += 128) {
-            uint32_t k[4];
-            load4(src, vec, i0 + lane * 4, wend, k);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                gt += k[u] > theta;
-                eq += k[u] == theta && i0 + lane * 4 + u < wend;
-            }
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        gt += __shfl_xor_sync(0xffffffffu, gt, o);
-        eq += __shfl_xor_sync(0xffffffffu, eq, o);
-    }
-    if (lane == 0) {
-        sh.warp_gt[warp] = gt;
-        sh.warp_eq[warp] = eq;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        int g = 0, e = 0;
-        for (int w = 0; w < kTopkWarps; ++w) {
-            g += sh.warp_gt[w];
-            e += sh.warp_eq[w];
-        }
-        sh.cta_gt = g;
-        sh.cta_eq = e;
-    }
-    cluster.sync();
-    if (tid == 0) {
-        // tie quota and output offset of every CTA, in rank (= position) order
-        int cgt[kMaxCluster], ceq[kMaxCluster];
-#pragma unroll
-        for (int rr = 0; rr < kMaxCluster; ++rr) {
-            const TopkShared* o = cluster.map_shared_rank(&sh, rr < CS ? rr : 0);
-            cgt[rr] = rr < CS ? o->cta_gt : 0;
-            ceq[rr] = rr < CS ? o->cta_eq : 0;
-        }
-        int eq_before = 0, sel_before = 0, eq_run = 0, sel_total = 0;
-#pragma unroll
-        for (int rr = 0; rr < kMaxCluster; ++rr) {
-            int take = krem - eq_run;
-            take = take < 0 ? 0 : (take > ceq[rr] ? ceq[rr] : take);
-            if (rr == rank) {
-                eq_before = eq_run;
-                sel_before = sel_total;
-            }
-            eq_run += ceq[rr];
-            sel_total += cgt[rr] + take;
-        }
-        int e = eq_before, s = sel_before;
-        for (int w = 0; w < kTopkWarps; ++w) {
-            sh.warp_eq_before[w] = e;
-            sh.warp_sel_before[w] = s;
-            int take = krem - e;
-            take = take < 0 ? 0 : (take > sh.warp_eq[w] ? sh.warp_eq[w] : take);
-            s += sh.warp_gt[w] + take;
-            e += sh.warp_eq[w];
-        }
-        sh.total = sel_total;
-    }
-    __syncthreads();
+    // uniform over the cluster: every CTA read the same counts
+    const bool fast = !any_over && (take_all || ncand_all <= kGatherCap);
 
     int32_t* out = a.idx + (size_t)row * a.B;
     const int32_t* bm = a.blkmap ? a.blkmap + (size_t)row * a.keep : nullptr;
-    const int eq_before = sh.warp_eq_before[warp];
-    int sel_pos = sh.warp_sel_before[warp];
-    int eq_seen = 0;
     const unsigned lt_mask = (1u << lane) - 1u;
+    uint32_t theta = 0;
+    int eq_before = 0, sel_pos = 0, eq_seen = 0;
     auto emit = [&](bool in, uint32_t k, int c) {
         const bool is_eq = in && k == theta;
         const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
@@ -474,13 +342,208 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkAr
         eq_seen += __popc(eqm);
         sel_pos += __popc(sm);
     };
-    if (!any_over) {
+    // per-warp counts of keys above / at theta, reduced into sh.warp_gt / warp_eq
+    auto warp_counts = [&](int gt, int eq) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            gt += __shfl_xor_sync(0xffffffffu, gt, o);
+            eq += __shfl_xor_sync(0xffffffffu, eq, o);
+        }
+        if (lane == 0) {
+            sh.warp_gt[warp] = gt;
+            sh.warp_eq[warp] = eq;
+        }
+        __syncthreads();
+    };
+    // warp offsets from this CTA's tie base and output base (thread 0)
+    auto warp_offsets = [&](int e, int s_) {
+        for (int w = 0; w < kTopkWarps; ++w) {
+            sh.warp_eq_before[w] = e;
+            sh.warp_sel_before[w] = s_;
+            int take = krem - e;
+            take = take < 0 ? 0 : (take > sh.warp_eq[w] ? sh.warp_eq[w] : take);
+            s_ += sh.warp_gt[w] + take;
+            e += sh.warp_eq[w];
+        }
+    };
+
+    if (fast) {
+        // ---- 3. theta from the cluster's bin-b0 keys, gathered into every CTA
+        int eq_rank = 0, sel_rank = 0, sel_total = 0;
+        if (!take_all) {
+            constexpr int kG = kGatherCap / kTopkThreads;
+            uint32_t v[kG];
+#pragma unroll
+            for (int u = 0; u < kG; ++u) {
+                const int i = u * kTopkThreads + tid;
+                int rr = 0;
+#pragma unroll
+                for (int q = 1; q < kMaxCluster; ++q) rr += i >= pre[q];
+                v[u] = i < ncand_all ? cluster.map_shared_rank(sh.cand, rr)[i - pre[rr]] : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kG; ++u) {
+                const int i = u * kTopkThreads + tid;
+                if (i < ncand_all) sh.gathered[i] = v[u];
+            }
+            // both local histograms (bits 10..20 in hist, bits 0..9 in red, whose
+            // row histogram is no longer needed) are cleared up front
+            for (int i = tid; i < kBins; i += kTopkThreads) sh.hist[i] = 0;
+            for (int i = tid; i < 1024; i += kTopkThreads) sh.red[i] = 0;
+            if (tid < 2 * kMaxCluster) sh.rcnt[tid] = 0;
+            __syncthreads();
+            uint32_t prefix = b0 << 21;
+            for (int i = tid; i < ncand_all; i += kTopkThreads)
+                atomicAdd(&sh.hist[(sh.gathered[i] >> 10) & 2047u], 1u);
+            __syncthreads();
+            find_bin(sh.hist, 2048, krem, sh);
+            prefix |= sh.bstar << 10;
+            krem -= sh.above;
+            for (int i = tid; i < ncand_all; i += kTopkThreads) {
+                const uint32_t k = sh.gathered[i];
+                if ((k & 0xfffffc00u) == prefix) atomicAdd(&sh.red[k & 1023u], 1u);
+            }
+            __syncthreads();
+            find_bin(sh.red, 1024, krem, sh);
+            prefix |= sh.bstar;
+            krem -= sh.above;
+            theta = prefix;
+            // per-rank counts above / at theta among the gathered keys (rank ranges)
+            for (int i = tid; i < ncand_all; i += kTopkThreads) {
+                int rr = 0;
+#pragma unroll
+                for (int q = 1; q < kMaxCluster; ++q) rr += i >= pre[q];
+                const uint32_t k = sh.gathered[i];
+                if (k > theta) atomicAdd(&sh.rcnt[rr], 1);
+                else if (k == theta) atomicAdd(&sh.rcnt[kMaxCluster + rr], 1);
+            }
+            __syncthreads();
+            int eq_run = 0, sel_run = 0;
+#pragma unroll
+            for (int rr = 0; rr < kMaxCluster; ++rr) {
+                if (rr < CS) {
+                    const int req = sh.rcnt[kMaxCluster + rr];
+                    int take = krem - eq_run;
+                    take = take < 0 ? 0 : (take > req ? req : take);
+                    if (rr == rank) {
+                        eq_rank = eq_run;
+                        sel_rank = sel_run;
+                    }
+                    eq_run += req;
+                    sel_run += (nl[rr] - cnt[rr]) + sh.rcnt[rr] + take;
+                }
+            }
+            sel_total = sel_run;
+        } else {
+            krem = 0;   // every valid key (key > 0 = theta) is taken
+            int sel_run = 0;
+#pragma unroll
+            for (int rr = 0; rr < kMaxCluster; ++rr) {
+                if (rr == rank) sel_rank = sel_run;
+                sel_run += nl[rr];   // zero for rr >= CS
+            }
+            sel_total = sel_run;
+        }
+        // ---- 4. counts over this warp's list, offsets, compaction of the list
+        int gt = 0, eq = 0;
+        for (int j = lane; j < wc; j += 32) {
+            const uint32_t k = wkey[j];
+            gt += k > theta;
+            eq += k == theta;
+        }
+        warp_counts(gt, eq);
+        if (tid == 0) {
+            warp_offsets(eq_rank, sel_rank);
+            sh.total = sel_total;
+        }
+        __syncthreads();
+        eq_before = sh.warp_eq_before[warp];
+        sel_pos = sh.warp_sel_before[warp];
         for (int j0 = 0; j0 < wc; j0 += 32) {
             const int j = j0 + lane;
             const bool in = j < wc;
             emit(in, in ? wkey[j] : 0u, in ? wpos[j] : 0);
         }
     } else {
+        // ---- 3'. too many keys for shared memory: resolve the low 21 bits with
+        // cluster-wide radix passes over the keys themselves
+        if (!take_all) {
+            uint32_t prefix = b0 << 21, pmask = 0xffe00000u;
+            for (int pass = 1; pass < 3; ++pass) {
+                const int shift = pass == 1 ? 10 : 0;
+                const int nb = pass == 1 ? 2048 : 1024;
+                for (int i = tid; i < nb; i += kTopkThreads) sh.hist[i] = 0;
+                __syncthreads();
+                for (int i0 = wbeg; i0 < wend; i0 += 128) {
+                    uint32_t k[4];
+                    load4(src, vec, i0 + lane * 4, wend, k);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (k[u] && (k[u] & pmask) == prefix)
+                            atomicAdd(&sh.hist[(k[u] >> shift) & (uint32_t)(nb - 1)], 1u);
+                }
+                cluster.sync();
+                cluster_reduce(cluster, sh.hist, sh.red, nb, CS);
+                cluster.sync();   // hist may be reset next pass only after every CTA has read it
+                find_bin(sh.red, nb, krem, sh);
+                prefix |= sh.bstar << shift;
+                pmask |= (uint32_t)(nb - 1) << shift;
+                krem -= sh.above;
+                __syncthreads();
+            }
+            theta = prefix;
+        } else {
+            krem = 0;
+        }
+        // ---- 4'. counts over the keys, cluster exchange, compaction of the keys
+        int gt = 0, eq = 0;
+        for (int i0 = wbeg; i0 < wend; i0 += 128) {
+            uint32_t k[4];
+            load4(src, vec, i0 + lane * 4, wend, k);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                gt += k[u] > theta;
+                eq += k[u] == theta && i0 + lane * 4 + u < wend;
+            }
+        }
+        warp_counts(gt, eq);
+        if (tid == 0) {
+            int g = 0, e = 0;
+            for (int w = 0; w < kTopkWarps; ++w) {
+                g += sh.warp_gt[w];
+                e += sh.warp_eq[w];
+            }
+            sh.cta_gt = g;
+            sh.cta_eq = e;
+        }
+        cluster.sync();
+        if (tid == 0) {
+            // tie quota and output offset of every CTA, in rank (= position) order
+            int cgt[kMaxCluster], ceq[kMaxCluster];
+#pragma unroll
+            for (int rr = 0; rr < kMaxCluster; ++rr) {
+                const TopkShared* o = cluster.map_shared_rank(&sh, rr < CS ? rr : 0);
+                cgt[rr] = rr < CS ? o->cta_gt : 0;
+                ceq[rr] = rr < CS ? o->cta_eq : 0;
+            }
+            int e0 = 0, s0 = 0, eq_run = 0, sel_total = 0;
+#pragma unroll
+            for (int rr = 0; rr < kMaxCluster; ++rr) {
+                int take = krem - eq_run;
+                take = take < 0 ? 0 : (take > ceq[rr] ? ceq[rr] : take);
+                if (rr == rank) {
+                    e0 = eq_run;
+                    s0 = sel_total;
+                }
+                eq_run += ceq[rr];
+                sel_total += cgt[rr] + take;
+            }
+            warp_offsets(e0, s0);
+            sh.total = sel_total;
+        }
+        __syncthreads();
+        eq_before = sh.warp_eq_before[warp];
+        sel_pos = sh.warp_sel_before[warp];
         for (int i0 = wbeg; i0 < wend; i0 += 32) {
             const int i = i0 + lane;
             const bool in = i < wend;
@@ -522,15 +585,16 @@ cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int
     cfg.blockDim = dim3(kTopkThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = ctx.stream;
-    cudaLaunchAttribute attr[2];
+    // Launched without programmatic dependent launch: placing 8-CTA clusters
+    // while the scorer's CTAs drain fragments the GPCs and pushed the last
+    // clusters into a second wave (measured); a plain launch places them all.
+    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
