@@ -61,7 +61,9 @@ enum {
     LSA_ERR_WORKSPACE = -4,   /* workspace missing, misaligned (256 B) or too small */
     LSA_ERR_CUDA = -5,        /* a CUDA launch failed (cudaGetLastError) */
     LSA_ERR_TIMEOUT = -6,     /* reserved: device-side bounded wait ran out (status word) */
-    LSA_ERR_UNSUPPORTED = -7  /* sizes outside the supported set above */
+    LSA_ERR_UNSUPPORTED = -7, /* sizes outside the supported set above */
+    LSA_ERR_SCRATCH = -8      /* sizes need more than the fixed scratch of
+                                 lsa_indexed_attn_noalloc holds */
 };
 
 /* Bits of the device status word (lsa_read_device_status). */
@@ -125,6 +127,43 @@ LSA_API lsa_status lsa_topk(const lsa_dims* dims, const float* scores, int B, in
 LSA_API lsa_status lsa_indexed_attn(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* k,
                             const lsa_bf16* v, const int32_t* idx, int B, float scale,
                             lsa_bf16* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of the fixed per-device scratch buffer of lsa_indexed_attn_noalloc. */
+#define LSA_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/* lsa_indexed_attn without a workspace, for callers that cannot allocate
+ * device memory where they make the call: a host thread that must not call
+ * cudaMalloc/cudaFree (both can synchronize the whole device and stall other
+ * streams), or code inside a framework that owns all device memory and hands
+ * out no scratch. The papers have no counterpart of this call; it is a
+ * deployment convenience around the same attention kernel.
+ * Arguments, supported sizes and results are those of lsa_indexed_attn,
+ * except:
+ *   - The split-softmax partials and merge counters live in one buffer of
+ *     LSA_NOALLOC_SCRATCH_BYTES per device inside liblsa.so. The library
+ *     allocates nothing: no cudaMalloc, no cudaFree, no allocating routine.
+ *   - Sizes that need more than that buffer return LSA_ERR_SCRATCH and launch
+ *     nothing. Every size with
+ *       batch * hkv * (4 + G * ceil(B / 64) * (d + 2) * 4) + 768
+ *         <= LSA_NOALLOC_SCRATCH_BYTES
+ *     is accepted (batch 4, hkv 8, G 4, d 128, B 2048 needs at most 2.2 MB);
+ *     larger ones often fit as well, since the split uses fewer slots.
+ *   - dev_status: NULL, or a caller-owned device int32 (4-byte aligned) into
+ *     which the LSA_DEV_* bits are OR-ed; the caller zeroes it.
+ *   - The first call on each device (the device current at the call) does a
+ *     one-time setup: it looks up the buffer's device address, zero-fills the
+ *     buffer on `stream` and waits for `stream`. Make that first call before
+ *     any stream capture begins; a first call on a capturing stream returns
+ *     LSA_ERR_CUDA and enqueues nothing.
+ *   - Only the merge counters at the start of the buffer must be zero when a
+ *     call starts; the setup zeroes them and every completed call leaves
+ *     them at zero. The partials need no initial value.
+ *   - All calls on one device share the buffer, so calls that overlap on the
+ *     GPU (unordered streams, concurrent host threads) race and produce wrong
+ *     outputs. Order them, e.g. on one stream. */
+LSA_API lsa_status lsa_indexed_attn_noalloc(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* k,
+                                    const lsa_bf16* v, const int32_t* idx, int B, float scale,
+                                    lsa_bf16* out, int32_t* dev_status, void* stream);
 
 /* One whole decode step: scoring, top-B and indexed attention (JSSA, Fig. 1).
  *   q [batch, hq, d], qt [batch, hq, r], k/v [batch, T, hkv, d],

@@ -22,7 +22,9 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "lsa.h")
 
 LSA_OK = 0
 STATUS_NAMES = {0: "LSA_OK", -1: "LSA_ERR_ARG", -2: "LSA_ERR_ALIGN", -3: "LSA_ERR_SHAPE",
-                -4: "LSA_ERR_WORKSPACE", -5: "LSA_ERR_CUDA", -6: "LSA_ERR_TIMEOUT", -7: "LSA_ERR_UNSUPPORTED"}
+                -4: "LSA_ERR_WORKSPACE", -5: "LSA_ERR_CUDA", -6: "LSA_ERR_TIMEOUT", -7: "LSA_ERR_UNSUPPORTED",
+                -8: "LSA_ERR_SCRATCH"}
+NOALLOC_SCRATCH_BYTES = 8 << 20   # LSA_NOALLOC_SCRATCH_BYTES
 DEV_BAD_INDEX = 1
 DEV_TIMEOUT = 2
 
@@ -52,6 +54,7 @@ _SIGS = {
     "lsa_score": (_I, [_DIMS, _P, _P, _P, _P]),
     "lsa_topk": (_I, [_DIMS, _P, _I, _P, _P, _SZ, _P]),
     "lsa_indexed_attn": (_I, [_DIMS, _P, _P, _P, _P, _I, ctypes.c_float, _P, _P, _SZ, _P]),
+    "lsa_indexed_attn_noalloc": (_I, [_DIMS, _P, _P, _P, _P, _I, ctypes.c_float, _P, _P, _P]),
     "lsa_decode_step": (_I, [_DIMS, _P, _P, _P, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _P, _SZ, _P]),
     "lsa_block_centroids": (_I, [_DIMS, _P, _I, _P, _P]),
     "lsa_prefill_workspace_size": (_SZ, [_DIMS, _I, _I]),
@@ -183,6 +186,29 @@ def lsa_indexed_attn(q, k, v, idx, scale: float | None = None, out=None, ws=None
     _check("lsa_indexed_attn", lib().lsa_indexed_attn(
         ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), int(B), ctypes.c_float(scale), _ptr(out),
         _ptr(ws), ws.numel(), _stream(q)))
+    return out
+
+
+def lsa_indexed_attn_noalloc(q, k, v, idx, scale: float | None = None, out=None, dev_status=None) -> torch.Tensor:
+    """lsa_indexed_attn with the library's fixed per-device scratch instead of a
+    workspace (lsa.h: lsa_indexed_attn_noalloc). dev_status: optional device
+    int32 [1] receiving LSA_DEV_* bits."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _cuda(t, n, torch.bfloat16)
+    _cuda(idx, "idx", torch.int32)
+    batch, hq, d = q.shape
+    _, T, hkv, _ = k.shape
+    B = idx.shape[-1]
+    dims = make_dims(batch, hq, hkv, d, 16, T)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    _cuda(out, "out", torch.bfloat16)
+    if dev_status is not None:
+        _cuda(dev_status, "dev_status", torch.int32)
+    _check("lsa_indexed_attn_noalloc", lib().lsa_indexed_attn_noalloc(
+        ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), int(B), ctypes.c_float(scale), _ptr(out),
+        _ptr(dev_status), _stream(q)))
     return out
 
 

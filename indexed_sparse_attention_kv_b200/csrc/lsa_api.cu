@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/lsa.h"
 #include "lsa_internal.h"
@@ -123,6 +124,40 @@ T* at(void* ws, size_t off) {
 
 }  // namespace
 
+// Scratch of lsa_indexed_attn_noalloc: one fixed buffer per device, part of
+// this module's device image, so that the call never allocates. Byte layout
+// of one call: merge counters [units] uint32 at offset 0 (zero between
+// calls), then pm, pl [slots] fp32 and po [slots, d] fp32, each 256-aligned.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LSA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch on the current device. The first call per
+// device looks it up and zero-fills the buffer on `stream`, waiting for it.
+lsa_status noalloc_scratch(cudaStream_t stream, void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LSA_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+            return LSA_ERR_CUDA;
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LSA_ERR_CUDA;
+        if (cudaMemsetAsync(p, 0, LSA_NOALLOC_SCRATCH_BYTES, stream) != cudaSuccess) return LSA_ERR_CUDA;
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return LSA_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return LSA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int lsa_version(void) { return 100; }
@@ -137,6 +172,8 @@ const char* lsa_status_string(lsa_status s) {
         case LSA_ERR_CUDA: return "LSA_ERR_CUDA: a CUDA launch failed";
         case LSA_ERR_TIMEOUT: return "LSA_ERR_TIMEOUT: a device-side wait ran out";
         case LSA_ERR_UNSUPPORTED: return "LSA_ERR_UNSUPPORTED: sizes outside the supported set";
+        case LSA_ERR_SCRATCH:
+            return "LSA_ERR_SCRATCH: sizes need more than the fixed no-alloc scratch (LSA_NOALLOC_SCRATCH_BYTES)";
         default: return "LSA_ERR_UNKNOWN";
     }
 }
@@ -190,6 +227,33 @@ lsa_status lsa_indexed_attn(const lsa_dims* dims, const lsa_bf16* q, const lsa_b
                                       at<unsigned>(ws, L.counters), dims->batch, dims->hq, dims->hkv,
                                       dims->d, dims->T, (long long)dims->T * dims->hkv,
                                       at<unsigned>(ws, L.status)));
+}
+
+lsa_status lsa_indexed_attn_noalloc(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* k, const lsa_bf16* v,
+                                    const int32_t* idx, int B, float scale, lsa_bf16* out, int32_t* dev_status,
+                                    void* stream) {
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if ((s = check_B(B)) != LSA_OK) return s;
+    if (!q || !k || !v || !idx || !out) return LSA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(out)) return LSA_ERR_ALIGN;
+    if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0) return LSA_ERR_ALIGN;
+    if (!std::isfinite(scale)) return LSA_ERR_ARG;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    const int G = dims->hq / dims->hkv;
+    const lsa::AttnPlan plan = lsa::plan_attn(dims->batch, dims->hkv, G, B, dims->d, ctx.num_sms);
+    const size_t slots = (size_t)plan.units * plan.smax * G;
+    const size_t pm = align_up((size_t)plan.units * 4);
+    const size_t pl = pm + align_up(slots * 4);
+    const size_t po = pl + align_up(slots * 4);
+    const size_t need = po + align_up(slots * (size_t)dims->d * 4);
+    if (need > LSA_NOALLOC_SCRATCH_BYTES) return LSA_ERR_SCRATCH;
+    void* base = nullptr;
+    if ((s = noalloc_scratch(ctx.stream, &base)) != LSA_OK) return s;
+    return from_cuda(lsa::launch_attn(ctx, plan, q, k, v, idx, B, scale, out, at<float>(base, pm),
+                                      at<float>(base, pl), at<float>(base, po), at<unsigned>(base, 0),
+                                      dims->batch, dims->hq, dims->hkv, dims->d, dims->T,
+                                      (long long)dims->T * dims->hkv, reinterpret_cast<unsigned*>(dev_status)));
 }
 
 lsa_status lsa_decode_step(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* qt, const lsa_bf16* k,
