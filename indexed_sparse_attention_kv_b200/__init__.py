@@ -14,6 +14,11 @@ from ._lib import (  # noqa: F401
     lsa_decode_step,
     lsa_dims,
     lsa_indexed_attn,
+    lsa_indexed_attn_noalloc,
+    lsa_prefill_attn,
+    lsa_prefill_index,
+    lsa_prefill_workspace_size,
+    prefill_workspace,
     lsa_read_device_status,
     lsa_score,
     lsa_topk,

@@ -252,6 +252,65 @@ def lsa_block_centroids(kt: torch.Tensor, blk: int, centroids=None) -> torch.Ten
     return centroids
 
 
+def lsa_prefill_workspace_size(dims: lsa_dims, nq: int, B: int) -> int:
+    return int(lib().lsa_prefill_workspace_size(ctypes.byref(dims), int(nq), int(B)))
+
+
+def prefill_workspace(dims: lsa_dims, nq: int, B: int, device="cuda") -> torch.Tensor:
+    """A zeroed uint8 prefill workspace (256-byte aligned)."""
+    n = lsa_prefill_workspace_size(dims, nq, B)
+    if n == 0:
+        raise LsaError("lsa_prefill_workspace_size", -1, f"invalid sizes {dims} nq={nq} B={B}")
+    ws = torch.zeros(n + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    return ws[off:off + n]
+
+
+def prefill_dims(hq: int, kt: torch.Tensor, d: int = 128) -> lsa_dims:
+    T, hkv, r = kt.shape
+    return make_dims(1, hq, hkv, d, r, T)
+
+
+def lsa_prefill_index(qt, kt, q_start: int, B: int, idx=None, ws=None) -> torch.Tensor:
+    """Causal top-B index sets [nq, hkv, B] of queries qt [nq, hq, r] at positions
+    q_start .. q_start + nq - 1 over kt [T, hkv, r] (lsa.h: lsa_prefill_index)."""
+    _cuda(qt, "qt", torch.bfloat16)
+    _cuda(kt, "kt", torch.bfloat16)
+    nq, hq, _ = qt.shape
+    dims = prefill_dims(hq, kt)
+    if idx is None:
+        idx = torch.empty((nq, dims.hkv, B), dtype=torch.int32, device=qt.device)
+    _cuda(idx, "idx", torch.int32)
+    if ws is None:
+        ws = prefill_workspace(dims, nq, B, device=qt.device)
+    _check("lsa_prefill_index", lib().lsa_prefill_index(
+        ctypes.byref(dims), _ptr(qt), int(nq), int(q_start), _ptr(kt), int(B), _ptr(idx), _ptr(ws), ws.numel(),
+        _stream(qt)))
+    return idx
+
+
+def lsa_prefill_attn(q, k, v, idx, scale: float | None = None, out=None, ws=None) -> torch.Tensor:
+    """Indexed attention of every prefill query q [nq, hq, d] over k/v [T, hkv, d]
+    rows idx [nq, hkv, B] (lsa.h: lsa_prefill_attn)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _cuda(t, n, torch.bfloat16)
+    _cuda(idx, "idx", torch.int32)
+    nq, hq, d = q.shape
+    T, hkv, _ = k.shape
+    B = idx.shape[-1]
+    dims = make_dims(1, hq, hkv, d, 16, T)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    _cuda(out, "out", torch.bfloat16)
+    if ws is None:
+        ws = prefill_workspace(dims, nq, B, device=q.device)
+    _check("lsa_prefill_attn", lib().lsa_prefill_attn(
+        ctypes.byref(dims), _ptr(q), int(nq), _ptr(k), _ptr(v), _ptr(idx), int(B), ctypes.c_float(scale), _ptr(out),
+        _ptr(ws), ws.numel(), _stream(q)))
+    return out
+
+
 def lsa_read_device_status(ws: torch.Tensor) -> int:
     """Synchronously read the workspace's device status word (LSA_DEV_* bits)."""
     host = torch.zeros(1, dtype=torch.int32).pin_memory()

@@ -110,6 +110,40 @@ DecodeLayout decode_layout(const lsa_dims* d, int B, int blk, int keep, int num_
     return L;
 }
 
+// Prefill workspace: status header, attention merge counters (zero between
+// calls), then one region shared by the indexer's buffers and the attention
+// partials (the two calls run one after the other).
+constexpr int kPrefillMaxT = 1 << 18;
+
+struct PrefillLayout {
+    size_t status = 0;
+    size_t counters = 0;
+    size_t region = 0;
+    size_t pm = 0, pl = 0, po = 0;
+    size_t total = 0;
+    lsa::PrefillPlan P{};
+    lsa::AttnPlan A{};
+};
+
+PrefillLayout prefill_layout(const lsa_dims* d, int nq, int B, int num_sms) {
+    PrefillLayout L;
+    size_t off = kHeaderBytes;
+    L.counters = off;
+    off = align_up(off + (size_t)nq * d->hkv * 4);
+    L.region = off;
+    L.P = lsa::plan_prefill(d->hq, d->hkv, d->r, d->T, nq, B);
+    const size_t index_end = L.region + L.P.bytes;
+    const int G = d->hq / d->hkv;
+    L.A = lsa::plan_attn(nq, d->hkv, G, B, d->d, num_sms);
+    const size_t slots = (size_t)L.A.units * L.A.smax * G;
+    L.pm = L.region;
+    L.pl = L.pm + align_up(slots * 4);
+    L.po = L.pl + align_up(slots * 4);
+    const size_t attn_end = L.po + align_up(slots * (size_t)d->d * 4);
+    L.total = align_up(index_end > attn_end ? index_end : attn_end);
+    return L;
+}
+
 lsa_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
     if (!ws) return LSA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return LSA_ERR_WORKSPACE;
@@ -330,25 +364,42 @@ lsa_status lsa_block_centroids(const lsa_dims* dims, const lsa_bf16* kt, int blk
 }
 
 size_t lsa_prefill_workspace_size(const lsa_dims* dims, int nq, int B) {
-    (void)dims;
-    (void)nq;
-    (void)B;
-    return 0;
+    if (check_dims(dims) != LSA_OK || check_B(B) != LSA_OK || nq < 1 || dims->batch != 1) return 0;
+    return prefill_layout(dims, nq, B, device_sms()).total;
 }
 
 lsa_status lsa_prefill_index(const lsa_dims* dims, const lsa_bf16* qt, int nq, int q_start, const lsa_bf16* kt, int B,
                              int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
-    (void)dims; (void)qt; (void)nq; (void)q_start; (void)kt; (void)B; (void)idx; (void)ws; (void)ws_bytes;
-    (void)stream;
-    return LSA_ERR_UNSUPPORTED;
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if ((s = check_B(B)) != LSA_OK) return s;
+    if (!qt || !kt || !idx || nq < 1 || q_start < 0) return LSA_ERR_ARG;
+    if (dims->batch != 1 || (long long)q_start + nq > dims->T) return LSA_ERR_SHAPE;
+    if (dims->T > kPrefillMaxT) return LSA_ERR_UNSUPPORTED;
+    if (!aligned16(qt) || !aligned16(kt) || !aligned16(idx)) return LSA_ERR_ALIGN;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    const PrefillLayout L = prefill_layout(dims, nq, B, ctx.num_sms);
+    if ((s = check_ws(ws, ws_bytes, L.total)) != LSA_OK) return s;
+    return from_cuda(lsa::launch_prefill_index(ctx, L.P, qt, kt, dims->hq, dims->hkv, dims->r, dims->T, nq, q_start, B,
+                                               idx, at<uint8_t>(ws, L.region), at<unsigned>(ws, L.status)));
 }
 
 lsa_status lsa_prefill_attn(const lsa_dims* dims, const lsa_bf16* q, int nq, const lsa_bf16* k, const lsa_bf16* v,
                             const int32_t* idx, int B, float scale, lsa_bf16* out, void* ws, size_t ws_bytes,
                             void* stream) {
-    (void)dims; (void)q; (void)nq; (void)k; (void)v; (void)idx; (void)B; (void)scale; (void)out; (void)ws;
-    (void)ws_bytes; (void)stream;
-    return LSA_ERR_UNSUPPORTED;
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if ((s = check_B(B)) != LSA_OK) return s;
+    if (!q || !k || !v || !idx || !out || nq < 1) return LSA_ERR_ARG;
+    if (dims->batch != 1) return LSA_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(out)) return LSA_ERR_ALIGN;
+    if (!std::isfinite(scale)) return LSA_ERR_ARG;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    const PrefillLayout L = prefill_layout(dims, nq, B, ctx.num_sms);
+    if ((s = check_ws(ws, ws_bytes, L.total)) != LSA_OK) return s;
+    return from_cuda(lsa::launch_attn(ctx, L.A, q, k, v, idx, B, scale, out, at<float>(ws, L.pm), at<float>(ws, L.pl),
+                                      at<float>(ws, L.po), at<unsigned>(ws, L.counters), nq, dims->hq, dims->hkv,
+                                      dims->d, dims->T, 0, at<unsigned>(ws, L.status)));
 }
 
 lsa_status lsa_read_device_status(const void* ws, int32_t* host_flags, void* stream) {

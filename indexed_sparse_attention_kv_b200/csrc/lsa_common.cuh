@@ -1,6 +1,7 @@
 // Shared device helpers for the liblsa kernels (sm_100a).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 

@@ -89,4 +89,27 @@ cudaError_t launch_attn(const LaunchCtx& ctx, const AttnPlan& plan, const uint16
                         float* po, unsigned* counters, int nb, int hq, int hkv, int d, int T,
                         long long kv_bstride_rows, unsigned* status);
 
+// Prefill indexer plan: sample stride, selection constants and the byte
+// offsets of its buffers inside the caller's workspace region.
+struct PrefillPlan {
+    int nq_pad;              // nq rounded up to the 128-row tile
+    long long rows;          // nq * hkv output rows
+    int S;                   // sample stride (key columns)
+    int kth;                 // rank of the sampled threshold
+    int cap;                 // candidate capacity per row
+    bool sample;             // some row may need a threshold (T > cap)
+    int ncol_sample;         // 256-column tiles of the sample matrix
+    long long ld_samp;       // sample row stride (floats)
+    int stages;              // TMA pipeline stages of the score GEMM
+    int gemm_smem;           // dynamic shared memory of the score GEMM
+    size_t off_qb, off_samp, off_thr, off_cnt, off_cand, bytes;
+};
+
+PrefillPlan plan_prefill(int hq, int hkv, int r, int T, int nq, int B);
+
+// idx [nq, hkv, B]; ws: the plan's region (256-byte aligned, no initial value).
+cudaError_t launch_prefill_index(const LaunchCtx& ctx, const PrefillPlan& P, const uint16_t* qt, const uint16_t* kt,
+                                 int hq, int hkv, int r, int T, int nq, int q_start, int B, int32_t* idx, uint8_t* ws,
+                                 unsigned* status);
+
 }  // namespace lsa

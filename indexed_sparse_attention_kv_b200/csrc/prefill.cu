@@ -1,0 +1,775 @@
+// Prefill indexer: for every query row p of a prefill and every KV head h,
+// the top-B positions t <= p of s[p,h,t] = q_bar[p,h] . kt[t,h] (LongCat
+// Sparse Attention, Abstract: the Lightning Indexer's dense O(L^2) scoring;
+// Joint Subspace Sparse Attention for Efficient Long-Context Decoding, Fig. 1
+// for the group-mean query).
+//
+// The scores are never materialised. The score GEMM runs on the tensor cores
+// (tcgen05.mma, operands staged by TMA in 128-byte-swizzled shared memory,
+// fp32 accumulators in TMEM), twice:
+//   1. sample pass: only every S-th key column. A per-row radix select over
+//      those samples gives a threshold theta_row that about 1.75 B of the
+//      row's keys exceed;
+//   2. filter pass: all causal columns; the epilogue appends (key, position)
+//      of every score >= theta_row to a per-row candidate list.
+// A final per-row selection takes the exact top B of the candidates (ties:
+// lower position) and writes them in ascending order through a position
+// bitmap. Rows whose list overflowed its capacity or holds fewer than B keys
+// (a sample that misjudged the row) are re-done exactly from scratch by the
+// same kernel, recomputing scores on the CUDA cores.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "lsa_common.cuh"
+#include "lsa_internal.h"
+
+namespace lsa {
+namespace {
+
+constexpr int kBM = 128;              // query rows per tile = TMEM lanes
+constexpr int kBN = 256;              // key columns per tile = fp32 TMEM columns
+constexpr int kGemmThreads = 384;     // warp 0 TMA, warp 1 MMA + TMEM owner, warps 4..11 epilogue
+constexpr int kEpiWarp0 = 4;
+constexpr int kEpiWarps = 8;
+constexpr int kAccCols = 2 * kBN;     // two accumulators (double-buffered)
+constexpr int kMaxStages = 4;
+constexpr int kSelThreads = 256;
+constexpr int kMaxSamples = 8192;
+constexpr int kModeSample = 0;        // epilogue writes scores of sampled columns
+constexpr int kModeFilter = 1;        // epilogue appends scores above the row threshold
+
+// tcgen05.mma instruction descriptor, kind::f16: D fp32, A and B bf16, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
+                            ((uint32_t)(kBM >> 4) << 24);
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Arrive once on `bar` when every tcgen05 operation this thread issued so far
+// has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes (lane i of the
+// warp gets TMEM lane base + i). The registers are valid after tmem_wait.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+}
+// Wait for this thread's TMEM loads; the registers are tied to the wait so
+// that no use of them is scheduled before it.
+__device__ __forceinline__ void tmem_wait(uint32_t (&v)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+                   "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),
+                   "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
+                   "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]),
+                   "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
+                 :
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand tile in the swizzled
+// layout TMA writes: rows of `rb` bytes (32, 64 or 128 = the swizzle span),
+// 8-row atoms `8 * rb` bytes apart.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t rb) {
+    const uint32_t layout = rb == 128 ? 2u : (rb == 64 ? 4u : 6u);
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) |
+           ((uint64_t)(((8u * rb) >> 4) & 0x3FFFu) << 32) | ((uint64_t)1u << 46) | ((uint64_t)layout << 61);
+}
+
+// ---------------------------------------------------------------- arguments
+struct GemmArgs {
+    int r, hkv, nq, nq_pad, q_start;
+    int rb_per_head;       // nq_pad / 128
+    int ncol_tiles;        // column tiles of the longest row
+    int S;                 // key stride of the B operand's rows (sample stride, or 1)
+    int stages;
+    long long ntiles;      // hkv * ncol_tiles * rb_per_head
+    float* samp;           // sample mode: [rows, ld_samp] fp32
+    long long ld_samp;
+    const uint32_t* thr;   // filter mode: [rows] order-key thresholds
+    unsigned* cnt;         // [rows] candidate counts (zero on entry)
+    uint2* cand;           // [rows, cap] (key, position)
+    int cap;
+    unsigned* status;
+    long long wait_limit;
+};
+
+struct TileCoord {
+    int h, c, rb;
+    bool active;
+};
+
+// Tiles are ordered head-major, then column tile, then row block, so that the
+// CTAs working at one time share the same key tile through L2.
+__device__ __forceinline__ TileCoord decode_tile(long long t, const GemmArgs& a) {
+    TileCoord tc;
+    tc.rb = (int)(t % a.rb_per_head);
+    const long long rest = t / a.rb_per_head;
+    tc.c = (int)(rest % a.ncol_tiles);
+    tc.h = (int)(rest / a.ncol_tiles);
+    const int qlast = min(tc.rb * kBM + kBM - 1, a.nq - 1);
+    const long long pmax = (long long)a.q_start + qlast;
+    tc.active = (long long)tc.c * kBN * a.S <= pmax;
+    return tc;
+}
+
+// ---------------------------------------------------------------- score GEMM
+// D[128 queries, 256 keys] = Qbar_h[rows] . Kt_h[cols]^T per tile, K = r.
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    prefill_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const GemmArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rb = a.r * 2 < 128 ? (uint32_t)a.r * 2 : 128u;   // bytes per row in one swizzle atom
+    const int atoms = a.r * 2 / (int)rb;
+    const uint32_t a_bytes = (uint32_t)kBM * a.r * 2, st_bytes = (uint32_t)(kBM + kBN) * a.r * 2;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + a.stages * st_bytes);
+    uint64_t* empty = full + kMaxStages;
+    uint64_t* tfull = empty + kMaxStages;
+    uint64_t* tempty = tfull + 2;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < a.stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], kEpiWarps);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tslot, kAccCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tslot;
+
+    auto fail = [&]() {
+        set_status(a.status, kStatusTimeout);
+        *abort_flag = 1;
+    };
+
+    // Every role loop is warp-uniform: lane 0 waits on the barrier and
+    // broadcasts the outcome, lane 0 issues, the warp moves on together.
+    auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait_bounded(bar, parity, a.wait_limit, abort_flag) ? 1 : 0;
+        return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    };
+
+    if (warp == 0) {   // ----------------------------------------------- TMA producer
+        int it = 0;
+        for (long long t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
+            const TileCoord tc = decode_tile(t, a);
+            if (!tc.active) continue;
+            const int s = it % a.stages;
+            const uint32_t ph = (uint32_t)(it / a.stages) & 1u;
+            if (!warp_wait(&empty[s], ph ^ 1u)) {
+                if (lane == 0) fail();
+                break;
+            }
+            if (lane == 0) {
+                uint8_t* As = sm + s * st_bytes;
+                uint8_t* Bs = As + a_bytes;
+                mbar_arrive_expect_tx(&full[s], st_bytes);
+                for (int at = 0; at < atoms; ++at) {
+                    tma_load_2d(As + at * kBM * rb, &tmA, at * 64, tc.h * a.nq_pad + tc.rb * kBM, &full[s]);
+                    tma_load_2d(Bs + at * kBN * rb, &tmB, tc.h * a.r + at * 64, tc.c * kBN, &full[s]);
+                }
+            }
+            __syncwarp();
+            ++it;
+        }
+    } else if (warp == 1) {   // ---------------------------------------- MMA issuer
+        const int nk = a.r / 16;
+        int it = 0, last_acc = -1;
+        uint32_t last_aph = 0;
+        for (long long t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
+            const TileCoord tc = decode_tile(t, a);
+            if (!tc.active) continue;
+            const int s = it % a.stages;
+            const uint32_t ph = (uint32_t)(it / a.stages) & 1u;
+            const int acc = it & 1;
+            const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+            if (!warp_wait(&tempty[acc], aph ^ 1u) || !warp_wait(&full[s], ph)) {
+                if (lane == 0) fail();
+                break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t As = smem_addr(sm + s * st_bytes), Bs = As + a_bytes;
+                const uint32_t d = tbase + (uint32_t)(acc * kBN);
+                for (int k = 0; k < nk; ++k) {
+                    const uint32_t kb = (uint32_t)k * 32u;     // 16 bf16 of K per MMA
+                    const uint32_t atom = kb / rb, within = kb % rb;
+                    tc_mma(d, umma_desc(As + atom * kBM * rb + within, rb),
+                           umma_desc(Bs + atom * kBN * rb + within, rb), k > 0 ? 1u : 0u);
+                }
+                tc_commit(&empty[s]);
+                tc_commit(&tfull[acc]);
+            }
+            __syncwarp();
+            last_acc = acc;
+            last_aph = aph;
+            ++it;
+        }
+        // On an abort, let the last MMAs finish before TMEM is released.
+        if (lane == 0 && *abort_flag && last_acc >= 0)
+            mbar_wait_bounded(&tfull[last_acc], last_aph, a.wait_limit, nullptr);
+        __syncwarp();
+    } else if (warp >= kEpiWarp0) {   // ------------------------------- epilogue
+        const int ew = warp - kEpiWarp0;
+        const int quarter = warp & 3;   // TMEM lanes this warp may access
+        const int half = ew >> 2;       // column half of the tile
+        const int row_in = quarter * 32 + lane;
+        const float qnan = __int_as_float(0x7fc00000);
+        int it = 0;
+        for (long long t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
+            const TileCoord tc = decode_tile(t, a);
+            if (!tc.active) continue;
+            const int acc = it & 1;
+            const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+            if (!warp_wait(&tfull[acc], aph)) {
+                if (lane == 0) fail();
+                break;
+            }
+            tc_fence_after();
+            const int q = tc.rb * kBM + row_in;
+            const bool vrow = q < a.nq;
+            const int p = a.q_start + q;
+            const long long grow = (long long)q * a.hkv + tc.h;
+            const int col0 = tc.c * kBN + half * 128;
+            const uint32_t taddr = tbase + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * kBN + half * 128);
+            if (MODE == kModeSample) {
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t v[32];
+                    tmem_ld32(taddr + ch * 32, v);
+                    tmem_wait(v);
+                    if (vrow) {
+                        float* dst = a.samp + grow * a.ld_samp + col0 + ch * 32;
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const int c0 = col0 + ch * 32 + j;
+                            float4 f;
+                            f.x = (long long)(c0 + 0) * a.S <= p ? __uint_as_float(v[j + 0]) : qnan;
+                            f.y = (long long)(c0 + 1) * a.S <= p ? __uint_as_float(v[j + 1]) : qnan;
+                            f.z = (long long)(c0 + 2) * a.S <= p ? __uint_as_float(v[j + 2]) : qnan;
+                            f.w = (long long)(c0 + 3) * a.S <= p ? __uint_as_float(v[j + 3]) : qnan;
+                            *reinterpret_cast<float4*>(dst + j) = f;
+                        }
+                    }
+                }
+            } else {
+                const uint32_t thr = vrow ? __ldg(&a.thr[grow]) : 0xFFFFFFFFu;
+                int n = 0;
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t v[32];
+                    tmem_ld32(taddr + ch * 32, v);
+                    tmem_wait(v);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int tpos = col0 + ch * 32 + j;
+                        n += (tpos <= p && score_key(__uint_as_float(v[j])) >= thr) ? 1 : 0;
+                    }
+                }
+                unsigned w = 0;
+                if (n) w = atomicAdd(&a.cnt[grow], (unsigned)n);
+                if (__any_sync(0xffffffffu, n != 0)) {
+                    uint2* dst = a.cand + grow * a.cap;
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t v[32];
+                        tmem_ld32(taddr + ch * 32, v);
+                        tmem_wait(v);
+                        if (n) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                const int tpos = col0 + ch * 32 + j;
+                                const uint32_t key = score_key(__uint_as_float(v[j]));
+                                if (tpos <= p && key >= thr) {
+                                    if (w < (unsigned)a.cap) dst[w] = make_uint2(key, (uint32_t)tpos);
+                                    ++w;
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+            ++it;
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, kAccCols);
+    }
+}
+
+// ---------------------------------------------------------------- group mean
+// qb[h, q, c] = bf16(mean over the group of qt[q, h*G + g, c]); rows q >= nq zero.
+__global__ void prefill_qbar_kernel(const uint16_t* __restrict__ qt, uint16_t* __restrict__ qb, int nq, int nq_pad,
+                                    int hq, int hkv, int r) {
+    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long total = (long long)hkv * nq_pad * r;
+    if (e >= total) return;
+    const int c = (int)(e % r);
+    const long long rest = e / r;
+    const int q = (int)(rest % nq_pad);
+    const int h = (int)(rest / nq_pad);
+    const int G = hq / hkv;
+    float s = 0.f;
+    if (q < nq) {
+        const uint16_t* src = qt + ((long long)q * hq + (long long)h * G) * r + c;
+        for (int g = 0; g < G; ++g) s += __uint_as_float((uint32_t)src[(long long)g * r] << 16);
+        s *= 1.0f / (float)G;
+    }
+    qb[e] = f2bf(s);
+}
+
+// ---------------------------------------------------------------- selection
+struct SelArgs {
+    int hkv, nq, nq_pad, q_start, B, cap, r, S, kth;
+    long long ld_samp;
+    const float* samp;
+    uint32_t* thr;
+    unsigned* cnt;
+    const uint2* cand;
+    const uint16_t* qb;
+    const uint16_t* kt;
+    int32_t* idx;
+};
+
+struct SelShared {
+    uint32_t hist[2048];
+    int wtot[32];
+    int bin, above, eqc;
+};
+
+// Exclusive block-wide prefix sum of v (thread order); *total = the sum.
+template <int NT>
+__device__ __forceinline__ int block_excl_scan(int v, int* wtot, int* total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wtot[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+        int w = lane < NT / 32 ? wtot[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        if (lane < NT / 32) wtot[lane] = w;
+    }
+    __syncthreads();
+    const int before = wid ? wtot[wid - 1] : 0;
+    *total = wtot[NT / 32 - 1];
+    __syncthreads();
+    return before + x - v;
+}
+
+// Block-wide radix selection (11 + 11 + 10 bits) of the need-th largest
+// non-zero key among key_of(i), i in [0, count). Results, identical in every
+// thread: *theta = that key, *n_gt = keys above it, *n_eq = keys equal to it,
+// *total = non-zero keys. With fewer than `need` keys: theta = 0, n_gt = total.
+template <int NT, class F>
+__device__ void block_select(F key_of, int count, int need, SelShared& sh, uint32_t* theta, int* n_gt, int* n_eq,
+                             int* total) {
+    const int tid = threadIdx.x;
+    uint32_t prefix = 0, pmask = 0;
+    int rem = need, gt = 0, eqc = 0;
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nb = pass == 2 ? 1024 : 2048;
+        for (int i = tid; i < 2048; i += NT) sh.hist[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < count; i += NT) {
+            const uint32_t k = key_of(i);
+            if (k != 0u && (k & pmask) == prefix) atomicAdd(&sh.hist[(k >> shift) & (uint32_t)(nb - 1)], 1u);
+        }
+        __syncthreads();
+        const int per = nb / NT;
+        const int top = nb - 1 - tid * per;
+        int s = 0;
+        for (int j = 0; j < per; ++j) s += (int)sh.hist[top - j];
+        int tot = 0;
+        const int excl = block_excl_scan<NT>(s, sh.wtot, &tot);
+        if (pass == 0) {
+            *total = tot;
+            if (tot < need) {
+                *theta = 0u;
+                *n_gt = tot;
+                *n_eq = 0;
+                return;
+            }
+        }
+        if (excl < rem && rem <= excl + s) {
+            int c = excl;
+            for (int j = 0; j < per; ++j) {
+                const int b = top - j;
+                const int hb = (int)sh.hist[b];
+                if (c + hb >= rem) {
+                    sh.bin = b;
+                    sh.above = c;
+                    sh.eqc = hb;
+                    break;
+                }
+                c += hb;
+            }
+        }
+        __syncthreads();
+        const int b = sh.bin;
+        rem -= sh.above;
+        gt += sh.above;
+        eqc = sh.eqc;
+        prefix |= (uint32_t)b << shift;
+        pmask |= (uint32_t)(nb - 1) << shift;
+        __syncthreads();
+    }
+    *theta = prefix;
+    *n_gt = gt;
+    *n_eq = eqc;
+}
+
+// theta_row = the kth-largest sampled score of the row (rows short enough to
+// keep every key get the smallest key, 1); also zeroes the row's count.
+__global__ void __launch_bounds__(kSelThreads) prefill_threshold_kernel(const SelArgs a) {
+    __shared__ SelShared sh;
+    __shared__ uint32_t skeys[kMaxSamples];
+    const int row = blockIdx.x;
+    const int q = row / a.hkv;
+    const int p = a.q_start + q;
+    if (p + 1 <= a.cap || a.samp == nullptr) {
+        if (threadIdx.x == 0) {
+            a.thr[row] = 1u;
+            a.cnt[row] = 0u;
+        }
+        return;
+    }
+    const int ms = (int)min((long long)(p / a.S + 1), a.ld_samp);
+    const float* src = a.samp + (long long)row * a.ld_samp;
+    for (int i = threadIdx.x; i < ms; i += kSelThreads) skeys[i] = score_key(__ldcg(src + i));
+    __syncthreads();
+    uint32_t theta;
+    int gt, eq, total;
+    block_select<kSelThreads>([&](int i) { return skeys[i]; }, ms, a.kth, sh, &theta, &gt, &eq, &total);
+    if (threadIdx.x == 0) {
+        a.thr[row] = total >= a.kth ? theta : 1u;
+        a.cnt[row] = 0u;
+    }
+}
+
+// Exact top-B of one row (dynamic shared memory: a bitmap of the row's
+// positions, 4 * ceil((q_start + nq) / 32) bytes).
+__global__ void __launch_bounds__(kSelThreads) prefill_select_kernel(const SelArgs a) {
+    __shared__ SelShared sh;
+    __shared__ float sq[128];
+    extern __shared__ uint32_t bitmap[];
+    const int row = blockIdx.x;
+    const int q = row / a.hkv, h = row % a.hkv;
+    const int p = a.q_start + q;
+    const int n = p + 1;
+    const int need = min(a.B, n);
+    const unsigned count = __ldcg(&a.cnt[row]);
+    const bool fb = count > (unsigned)a.cap || count < (unsigned)need;
+    const uint2* cand = a.cand + (long long)row * a.cap;
+    const int r = a.r;
+    if (fb) {
+        for (int c = threadIdx.x; c < r; c += kSelThreads)
+            sq[c] = __uint_as_float((uint32_t)a.qb[((long long)h * a.nq_pad + q) * r + c] << 16);
+        __syncthreads();
+    }
+    // Scores recomputed on the CUDA cores (fallback rows only): fp32 FMAs over
+    // the r channels in order.
+    auto recompute = [&](int t) -> uint32_t {
+        const uint4* kr = reinterpret_cast<const uint4*>(a.kt + ((long long)t * a.hkv + h) * r);
+        float acc = 0.f;
+        for (int c8 = 0; c8 < r / 8; ++c8) {
+            const uint4 w = __ldg(kr + c8);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                acc = fmaf(sq[c8 * 8 + 2 * j], bf16lo(ws[j]), acc);
+                acc = fmaf(sq[c8 * 8 + 2 * j + 1], bf16hi(ws[j]), acc);
+            }
+        }
+        return score_key(acc);
+    };
+    auto key_of = [&](int i) -> uint32_t { return fb ? recompute(i) : __ldcg(&cand[i]).x; };
+    auto pos_of = [&](int i) -> uint32_t { return fb ? (uint32_t)i : __ldcg(&cand[i]).y; };
+    const int items = fb ? n : (int)count;
+
+    uint32_t theta;
+    int gt, eq, total;
+    block_select<kSelThreads>(key_of, items, need, sh, &theta, &gt, &eq, &total);
+    uint32_t pos_thr = 0xFFFFFFFFu;
+    if (theta != 0u && eq > need - gt) {
+        // Equal keys at the boundary: keep the need - gt lowest positions.
+        uint32_t th2;
+        int g2, e2, t2;
+        block_select<kSelThreads>(
+            [&](int i) -> uint32_t { return key_of(i) == theta ? ~pos_of(i) : 0u; }, items, need - gt, sh, &th2, &g2,
+            &e2, &t2);
+        pos_thr = ~th2;
+    }
+    const int nw = (n + 31) >> 5;
+    for (int w = threadIdx.x; w < nw; w += kSelThreads) bitmap[w] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < items; i += kSelThreads) {
+        const uint32_t k = key_of(i);
+        if (k == 0u) continue;
+        const uint32_t pos = pos_of(i);
+        if (k > theta || (k == theta && pos <= pos_thr)) atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
+    }
+    __syncthreads();
+    const int per = (nw + kSelThreads - 1) / kSelThreads;
+    const int w0 = min(nw, (int)threadIdx.x * per), w1 = min(nw, w0 + per);
+    int c = 0;
+    for (int w = w0; w < w1; ++w) c += __popc(bitmap[w]);
+    int nsel = 0;
+    int o = block_excl_scan<kSelThreads>(c, sh.wtot, &nsel);
+    int32_t* out = a.idx + (long long)row * a.B;
+    for (int w = w0; w < w1; ++w) {
+        uint32_t bits = bitmap[w];
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1u;
+            if (o < a.B) out[o] = w * 32 + b;
+            ++o;
+        }
+    }
+    for (int j = nsel + threadIdx.x; j < a.B; j += kSelThreads) out[j] = -1;
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor map: `outer` rows of `inner` elements, rows `row_bytes`
+// apart; boxes of box_inner x box_outer, swizzled to the box's row width.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+              uint32_t box_inner, uint32_t box_outer) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    const uint32_t bytes = box_inner * 2;
+    const CUtensorMapSwizzle sw = bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_32B;
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+}  // namespace
+
+PrefillPlan plan_prefill(int hq, int hkv, int r, int T, int nq, int B) {
+    PrefillPlan P{};
+    (void)hq;
+    P.nq_pad = (nq + kBM - 1) / kBM * kBM;
+    P.rows = (long long)nq * hkv;
+    // Sample stride: about 64 samples per B keys, at most kMaxSamples per row.
+    int S = 1;
+    while (S * 2 <= B / 64) S *= 2;
+    while (((long long)T + S - 1) / S > kMaxSamples) S *= 2;
+    P.S = S;
+    P.kth = (int)((3LL * B + 2LL * S - 1) / (2LL * S)) + 16;    // ceil(1.5 B / S) + 16
+    const long long expect = (long long)P.kth * S;               // keys expected above theta
+    long long cap = 2 * expect;
+    if (cap < B + B / 2 + 512) cap = B + B / 2 + 512;
+    P.cap = (int)((cap + 255) / 256 * 256);
+    P.sample = T > P.cap;
+    const long long m = ((long long)T + S - 1) / S;
+    P.ncol_sample = (int)((m + kBN - 1) / kBN);
+    P.ld_samp = (long long)P.ncol_sample * kBN;
+    const size_t st = (size_t)(kBM + kBN) * r * 2;
+    int stages = (int)((192 * 1024) / st);
+    if (stages > kMaxStages) stages = kMaxStages;
+    P.stages = stages;
+    size_t smem = stages * st + 2 * kMaxStages * 8 + 4 * 8 + 16 + 1024;
+    if (smem < 120 * 1024) smem = 120 * 1024;   // one CTA per SM: each holds all 512 TMEM columns
+    P.gemm_smem = (int)smem;
+    size_t off = 0;
+    P.off_qb = off;
+    off = align256(off + (size_t)hkv * P.nq_pad * r * 2);
+    P.off_samp = off;
+    if (P.sample) off = align256(off + (size_t)P.rows * P.ld_samp * 4);
+    P.off_thr = off;
+    off = align256(off + (size_t)P.rows * 4);
+    P.off_cnt = off;
+    off = align256(off + (size_t)P.rows * 4);
+    P.off_cand = off;
+    off = align256(off + (size_t)P.rows * P.cap * 8);
+    P.bytes = off;
+    return P;
+}
+
+cudaError_t launch_prefill_index(const LaunchCtx& ctx, const PrefillPlan& P, const uint16_t* qt, const uint16_t* kt,
+                                 int hq, int hkv, int r, int T, int nq, int q_start, int B, int32_t* idx, uint8_t* ws,
+                                 unsigned* status) {
+    uint16_t* qb = reinterpret_cast<uint16_t*>(ws + P.off_qb);
+    float* samp = P.sample ? reinterpret_cast<float*>(ws + P.off_samp) : nullptr;
+    uint32_t* thr = reinterpret_cast<uint32_t*>(ws + P.off_thr);
+    unsigned* cnt = reinterpret_cast<unsigned*>(ws + P.off_cnt);
+    uint2* cand = reinterpret_cast<uint2*>(ws + P.off_cand);
+
+    {
+        const long long total = (long long)hkv * P.nq_pad * r;
+        prefill_qbar_kernel<<<(unsigned)((total + 255) / 256), 256, 0, ctx.stream>>>(qt, qb, nq, P.nq_pad, hq, hkv, r);
+    }
+    CUtensorMap mA, mB, mS;
+    const uint32_t box_in = r < 64 ? (uint32_t)r : 64u;
+    if (!make_map(&mA, qb, (uint64_t)r, (uint64_t)hkv * P.nq_pad, (uint64_t)r * 2, box_in, kBM) ||
+        !make_map(&mB, kt, (uint64_t)hkv * r, (uint64_t)T, (uint64_t)hkv * r * 2, box_in, kBN))
+        return cudaErrorInvalidValue;
+    const long long nsamp_rows = ((long long)T + P.S - 1) / P.S;
+    if (P.sample &&
+        !make_map(&mS, kt, (uint64_t)hkv * r, (uint64_t)nsamp_rows, (uint64_t)hkv * r * 2 * P.S, box_in, kBN))
+        return cudaErrorInvalidValue;
+
+    GemmArgs g{};
+    g.r = r;
+    g.hkv = hkv;
+    g.nq = nq;
+    g.nq_pad = P.nq_pad;
+    g.q_start = q_start;
+    g.rb_per_head = P.nq_pad / kBM;
+    g.stages = P.stages;
+    g.thr = thr;
+    g.cnt = cnt;
+    g.cand = cand;
+    g.cap = P.cap;
+    g.status = status;
+    g.wait_limit = ctx.wait_limit;
+    const long long pmax = (long long)q_start + nq - 1;
+
+    SelArgs s{};
+    s.hkv = hkv;
+    s.nq = nq;
+    s.nq_pad = P.nq_pad;
+    s.q_start = q_start;
+    s.B = B;
+    s.cap = P.cap;
+    s.r = r;
+    s.S = P.S;
+    s.kth = P.kth;
+    s.ld_samp = P.ld_samp;
+    s.samp = samp;
+    s.thr = thr;
+    s.cnt = cnt;
+    s.cand = cand;
+    s.qb = qb;
+    s.kt = kt;
+    s.idx = idx;
+    const bool any_sample = P.sample && pmax + 1 > P.cap;
+
+    cudaError_t e;
+    if (any_sample) {
+        GemmArgs gs = g;
+        gs.S = P.S;
+        gs.ncol_tiles = (int)((pmax / P.S + 1 + kBN - 1) / kBN);
+        gs.ntiles = (long long)hkv * gs.ncol_tiles * gs.rb_per_head;
+        gs.samp = samp;
+        gs.ld_samp = P.ld_samp;
+        if ((e = ensure_dyn_smem((const void*)prefill_gemm_kernel<kModeSample>, P.gemm_smem)) != cudaSuccess) return e;
+        const unsigned grid = (unsigned)(gs.ntiles < ctx.num_sms ? gs.ntiles : ctx.num_sms);
+        prefill_gemm_kernel<kModeSample><<<grid, kGemmThreads, P.gemm_smem, ctx.stream>>>(mA, mS, gs);
+    } else {
+        s.samp = nullptr;
+    }
+    prefill_threshold_kernel<<<(unsigned)P.rows, kSelThreads, 0, ctx.stream>>>(s);
+    {
+        GemmArgs gf = g;
+        gf.S = 1;
+        gf.ncol_tiles = (int)((pmax + 1 + kBN - 1) / kBN);
+        gf.ntiles = (long long)hkv * gf.ncol_tiles * gf.rb_per_head;
+        if ((e = ensure_dyn_smem((const void*)prefill_gemm_kernel<kModeFilter>, P.gemm_smem)) != cudaSuccess) return e;
+        const unsigned grid = (unsigned)(gf.ntiles < ctx.num_sms ? gf.ntiles : ctx.num_sms);
+        prefill_gemm_kernel<kModeFilter><<<grid, kGemmThreads, P.gemm_smem, ctx.stream>>>(mA, mB, gf);
+    }
+    {
+        const int nw = (int)((pmax + 1 + 31) / 32);
+        const int smem = nw * 4;
+        if ((e = ensure_dyn_smem((const void*)prefill_select_kernel, smem)) != cudaSuccess) return e;
+        prefill_select_kernel<<<(unsigned)P.rows, kSelThreads, smem, ctx.stream>>>(s);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace lsa

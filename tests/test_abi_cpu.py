@@ -93,3 +93,37 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 4, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         L.lsa_score(q[:, :, :64], torch.zeros(1, 8, 1, 64, dtype=torch.bfloat16))
+
+
+def test_prefill_validation():
+    lib = L.lib()
+    d = _dims(T=4096)
+    assert lib.lsa_prefill_workspace_size(ctypes.byref(d), 256, 256) > 0
+    assert lib.lsa_prefill_workspace_size(ctypes.byref(_dims(batch=2)), 256, 256) == 0
+    assert lib.lsa_prefill_workspace_size(ctypes.byref(d), 0, 256) == 0
+    args = (ALIGNED, 256, 3840, ALIGNED, 256, ALIGNED, ALIGNED, 1 << 40, None)
+    assert lib.lsa_prefill_index(ctypes.byref(_dims(batch=2)), *args) == -3
+    assert lib.lsa_prefill_index(ctypes.byref(d), ALIGNED, 256, 3841, ALIGNED, 256, ALIGNED, ALIGNED, 1 << 40,
+                                 None) == -3
+    assert lib.lsa_prefill_index(ctypes.byref(d), ALIGNED, 0, 0, ALIGNED, 256, ALIGNED, ALIGNED, 1 << 40,
+                                 None) == -1
+    assert lib.lsa_prefill_index(ctypes.byref(_dims(T=(1 << 18) + 1)), *args) == -7
+    assert lib.lsa_prefill_index(ctypes.byref(d), MISALIGNED, 256, 3840, ALIGNED, 256, ALIGNED, ALIGNED, 1 << 40,
+                                 None) == -2
+    assert lib.lsa_prefill_index(ctypes.byref(d), ALIGNED, 256, 3840, ALIGNED, 256, ALIGNED, ALIGNED, 16,
+                                 None) == -4
+    f = ctypes.c_float
+    assert lib.lsa_prefill_attn(ctypes.byref(d), ALIGNED, 256, ALIGNED, ALIGNED, ALIGNED, 256, f(0.1), ALIGNED,
+                                ALIGNED, 16, None) == -4
+    assert lib.lsa_prefill_attn(ctypes.byref(d), ALIGNED, 256, ALIGNED, ALIGNED, ALIGNED, 256, f(float("nan")),
+                                ALIGNED, ALIGNED, 1 << 40, None) == -1
+
+
+def test_noalloc_rejects_before_any_device_use():
+    lib = L.lib()
+    d = L.make_dims(64, 128, 8, 256, 16, 1 << 17)
+    f = ctypes.c_float
+    assert lib.lsa_indexed_attn_noalloc(ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, ALIGNED, 65536, f(0.06),
+                                        ALIGNED, None, None) == -8
+    assert lib.lsa_indexed_attn_noalloc(ctypes.byref(d), MISALIGNED, ALIGNED, ALIGNED, ALIGNED, 16, f(0.06),
+                                        ALIGNED, None, None) == -2
