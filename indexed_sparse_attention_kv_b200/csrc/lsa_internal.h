@@ -101,6 +101,7 @@ struct PrefillPlan {
     int ncol_sample;         // 256-column tiles of the sample matrix
     long long ld_samp;       // sample row stride (floats)
     int stages;              // TMA pipeline stages of the score GEMM
+    int a_slots;             // query tiles in flight in the score GEMM (1 or 2)
     int gemm_smem;           // dynamic shared memory of the score GEMM
     size_t off_qb, off_samp, off_thr, off_cnt, off_cand, bytes;
 };

@@ -36,9 +36,12 @@ constexpr int kGemmThreads = 384;     // warp 0 TMA, warp 1 MMA + TMEM owner, wa
 constexpr int kEpiWarp0 = 4;
 constexpr int kEpiWarps = 8;
 constexpr int kAccCols = 2 * kBN;     // two accumulators (double-buffered)
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 6;
 constexpr int kSelThreads = 256;
 constexpr int kMaxSamples = 8192;
+constexpr int kMaxSlots = 8;
+constexpr int kStageRow = 36;         // staging row pitch (floats): conflict-free 16-byte stores
+constexpr int kStageFloats = 32 * kStageRow;          // writer slots per row (2 x at most 4 segments)
 constexpr int kModeSample = 0;        // epilogue writes scores of sampled columns
 constexpr int kModeFilter = 1;        // epilogue appends scores above the row threshold
 
@@ -121,44 +124,69 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t rb) {
 }
 
 // ---------------------------------------------------------------- arguments
+// Work is split into units (KV head h, 128-row block rb, column segment seg):
+// one CTA runs a unit's column tiles in order, so every output row has a
+// fixed set of writers: 2 * nseg threads (segment x tile half). Writer slot
+// = half * nseg + seg; slots 2j and 2j+1 share the j-th region of cap_pair
+// entries of the row's list, one filling it upward from the start, the other
+// downward from the end, so no writer needs an atomic. A pair whose two counts
+// add up to more than cap_pair has overflowed (the row is re-selected).
 struct GemmArgs {
     int r, hkv, nq, nq_pad, q_start;
-    int rb_per_head;       // nq_pad / 128
-    int ncol_tiles;        // column tiles of the longest row
+    int nrb;               // row blocks per head = nq_pad / 128
+    int ncol;              // column tiles of the longest row
+    int nseg;              // column segments per row block (1, 2 or 4)
     int S;                 // key stride of the B operand's rows (sample stride, or 1)
     int stages;
-    long long ntiles;      // hkv * ncol_tiles * rb_per_head
-    float* samp;           // sample mode: [rows, ld_samp] fp32
+    int a_slots;           // A tiles in flight (2 = the next unit's loads overlap this unit's MMAs)
+    int nunits;            // hkv * nseg * nrb
+    uint16_t* samp;        // sample mode: [rows, ld_samp] top 16 bits of the order keys (0 = none)
     long long ld_samp;
     const uint32_t* thr;   // filter mode: [rows] order-key thresholds
-    unsigned* cnt;         // [rows] candidate counts (zero on entry)
+    unsigned* cnt;         // [rows, 2 * nseg] per-writer counts
     uint2* cand;           // [rows, cap] (key, position)
-    int cap;
+    int cap_pair;          // entries per writer pair region
+    long long ld_cand;     // entries per row = nseg * cap_pair
     unsigned* status;
     long long wait_limit;
 };
 
-struct TileCoord {
-    int h, c, rb;
-    bool active;
+struct Unit {
+    int h, seg, rb;
+    int c0, c1;            // active column tiles [c0, c1)
+    long long pmin;        // position of the block's first query
 };
 
-// Tiles are ordered head-major, then column tile, then row block, so that the
-// CTAs working at one time share the same key tile through L2.
-__device__ __forceinline__ TileCoord decode_tile(long long t, const GemmArgs& a) {
-    TileCoord tc;
-    tc.rb = (int)(t % a.rb_per_head);
-    const long long rest = t / a.rb_per_head;
-    tc.c = (int)(rest % a.ncol_tiles);
-    tc.h = (int)(rest / a.ncol_tiles);
-    const int qlast = min(tc.rb * kBM + kBM - 1, a.nq - 1);
+// Units are ordered head, then segment, then row block: the CTAs running at
+// one time work through the same key columns of one head and share them in L2.
+__device__ __forceinline__ Unit decode_unit(int u, const GemmArgs& a) {
+    Unit t;
+    t.rb = u % a.nrb;
+    const int rest = u / a.nrb;
+    t.seg = rest % a.nseg;
+    t.h = rest / a.nseg;
+    const int qlast = min(t.rb * kBM + kBM - 1, a.nq - 1);
     const long long pmax = (long long)a.q_start + qlast;
-    tc.active = (long long)tc.c * kBN * a.S <= pmax;
-    return tc;
+    // the block's active tiles (those holding a column <= pmax), split evenly
+    const int act = (int)min((long long)a.ncol, pmax / ((long long)kBN * a.S) + 1);
+    t.c0 = (int)((long long)t.seg * act / a.nseg);
+    t.c1 = (int)((long long)(t.seg + 1) * act / a.nseg);
+    t.pmin = (long long)a.q_start + (long long)t.rb * kBM;
+    return t;
+}
+
+// Order key -> the smallest float with that key (keys of NaN patterns -> -inf),
+// so that s >= key_floor(k) <=> score_key(s) >= k for every non-NaN s.
+__device__ __forceinline__ float key_floor(uint32_t k) {
+    if (k & 0x80000000u) return __uint_as_float(k & 0x7FFFFFFFu);
+    if (k <= 0x007FFFFFu) return -__int_as_float(0x7f800000);
+    return __uint_as_float(~k);
 }
 
 // ---------------------------------------------------------------- score GEMM
 // D[128 queries, 256 keys] = Qbar_h[rows] . Kt_h[cols]^T per tile, K = r.
+// Shared memory: two A slots (one per unit, double-buffered), `stages` B
+// stages, barriers.
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -169,10 +197,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rb = a.r * 2 < 128 ? (uint32_t)a.r * 2 : 128u;   // bytes per row in one swizzle atom
     const int atoms = a.r * 2 / (int)rb;
-    const uint32_t a_bytes = (uint32_t)kBM * a.r * 2, st_bytes = (uint32_t)(kBM + kBN) * a.r * 2;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + a.stages * st_bytes);
+    const uint32_t a_bytes = (uint32_t)kBM * a.r * 2, b_bytes = (uint32_t)kBN * a.r * 2;
+    uint8_t* Aslot = sm;
+    uint8_t* Bst = sm + a.a_slots * a_bytes;
+    float* stage_all = reinterpret_cast<float*>(Bst + a.stages * b_bytes);   // epilogue staging, kStageFloats per warp
+    uint64_t* full = reinterpret_cast<uint64_t*>(stage_all + kEpiWarps * kStageFloats);
     uint64_t* empty = full + kMaxStages;
-    uint64_t* tfull = empty + kMaxStages;
+    uint64_t* afull = empty + kMaxStages;
+    uint64_t* aempty = afull + 2;
+    uint64_t* tfull = aempty + 2;
     uint64_t* tempty = tfull + 2;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
@@ -183,6 +216,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&afull[i], 1);
+            mbar_init(&aempty[i], 1);
             mbar_init(&tfull[i], 1);
             mbar_init(&tempty[i], kEpiWarps);
         }
@@ -202,7 +237,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         set_status(a.status, kStatusTimeout);
         *abort_flag = 1;
     };
-
     // Every role loop is warp-uniform: lane 0 waits on the barrier and
     // broadcasts the outcome, lane 0 issues, the warp moves on together.
     auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -212,61 +246,89 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     };
 
     if (warp == 0) {   // ----------------------------------------------- TMA producer
-        int it = 0;
-        for (long long t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
-            const TileCoord tc = decode_tile(t, a);
-            if (!tc.active) continue;
-            const int s = it % a.stages;
-            const uint32_t ph = (uint32_t)(it / a.stages) & 1u;
-            if (!warp_wait(&empty[s], ph ^ 1u)) {
-                if (lane == 0) fail();
+        int it = 0, ui = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < a.nunits && ok; u += gridDim.x) {
+            const Unit un = decode_unit(u, a);
+            if (un.c1 <= un.c0) continue;
+            const int as = ui % a.a_slots;
+            if (!warp_wait(&aempty[as], ((uint32_t)(ui / a.a_slots) & 1u) ^ 1u)) {
+                ok = false;
                 break;
             }
             if (lane == 0) {
-                uint8_t* As = sm + s * st_bytes;
-                uint8_t* Bs = As + a_bytes;
-                mbar_arrive_expect_tx(&full[s], st_bytes);
-                for (int at = 0; at < atoms; ++at) {
-                    tma_load_2d(As + at * kBM * rb, &tmA, at * 64, tc.h * a.nq_pad + tc.rb * kBM, &full[s]);
-                    tma_load_2d(Bs + at * kBN * rb, &tmB, tc.h * a.r + at * 64, tc.c * kBN, &full[s]);
-                }
+                mbar_arrive_expect_tx(&afull[as], a_bytes);
+                for (int at = 0; at < atoms; ++at)
+                    tma_load_2d(Aslot + as * a_bytes + at * kBM * rb, &tmA, at * 64, un.h * a.nq_pad + un.rb * kBM,
+                                &afull[as]);
             }
             __syncwarp();
-            ++it;
+            for (int c = un.c0; c < un.c1; ++c) {
+                const int s = it % a.stages;
+                const uint32_t ph = (uint32_t)(it / a.stages) & 1u;
+                if (!warp_wait(&empty[s], ph ^ 1u)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t* Bs = Bst + s * b_bytes;
+                    mbar_arrive_expect_tx(&full[s], b_bytes);
+                    for (int at = 0; at < atoms; ++at)
+                        tma_load_2d(Bs + at * kBN * rb, &tmB, un.h * a.r + at * 64, c * kBN, &full[s]);
+                }
+                __syncwarp();
+                ++it;
+            }
+            ++ui;
         }
+        if (!ok && lane == 0) fail();
     } else if (warp == 1) {   // ---------------------------------------- MMA issuer
         const int nk = a.r / 16;
-        int it = 0, last_acc = -1;
+        int it = 0, ui = 0, last_acc = -1;
         uint32_t last_aph = 0;
-        for (long long t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
-            const TileCoord tc = decode_tile(t, a);
-            if (!tc.active) continue;
-            const int s = it % a.stages;
-            const uint32_t ph = (uint32_t)(it / a.stages) & 1u;
-            const int acc = it & 1;
-            const uint32_t aph = (uint32_t)(it >> 1) & 1u;
-            if (!warp_wait(&tempty[acc], aph ^ 1u) || !warp_wait(&full[s], ph)) {
-                if (lane == 0) fail();
+        bool ok = true;
+        for (int u = blockIdx.x; u < a.nunits && ok; u += gridDim.x) {
+            const Unit un = decode_unit(u, a);
+            if (un.c1 <= un.c0) continue;
+            const int as = ui % a.a_slots;
+            if (!warp_wait(&afull[as], (uint32_t)(ui / a.a_slots) & 1u)) {
+                ok = false;
                 break;
             }
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t As = smem_addr(sm + s * st_bytes), Bs = As + a_bytes;
-                const uint32_t d = tbase + (uint32_t)(acc * kBN);
-                for (int k = 0; k < nk; ++k) {
-                    const uint32_t kb = (uint32_t)k * 32u;     // 16 bf16 of K per MMA
-                    const uint32_t atom = kb / rb, within = kb % rb;
-                    tc_mma(d, umma_desc(As + atom * kBM * rb + within, rb),
-                           umma_desc(Bs + atom * kBN * rb + within, rb), k > 0 ? 1u : 0u);
+            const uint32_t Asa = smem_addr(Aslot + as * a_bytes);
+            for (int c = un.c0; c < un.c1; ++c) {
+                const int s = it % a.stages;
+                const uint32_t ph = (uint32_t)(it / a.stages) & 1u;
+                const int acc = it & 1;
+                const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+                if (!warp_wait(&tempty[acc], aph ^ 1u) || !warp_wait(&full[s], ph)) {
+                    ok = false;
+                    break;
                 }
-                tc_commit(&empty[s]);
-                tc_commit(&tfull[acc]);
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t Bs = smem_addr(Bst + s * b_bytes);
+                    const uint32_t d = tbase + (uint32_t)(acc * kBN);
+                    for (int k = 0; k < nk; ++k) {
+                        const uint32_t kb = (uint32_t)k * 32u;     // 16 bf16 of K per MMA
+                        const uint32_t atom = kb / rb, within = kb % rb;
+                        tc_mma(d, umma_desc(Asa + atom * kBM * rb + within, rb),
+                               umma_desc(Bs + atom * kBN * rb + within, rb), k > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&empty[s]);
+                    tc_commit(&tfull[acc]);
+                }
+                __syncwarp();
+                last_acc = acc;
+                last_aph = aph;
+                ++it;
             }
+            if (!ok) break;
+            if (lane == 0) tc_commit(&aempty[as]);   // A slot free once this unit's MMAs are done
             __syncwarp();
-            last_acc = acc;
-            last_aph = aph;
-            ++it;
+            ++ui;
         }
+        if (!ok && lane == 0) fail();
         // On an abort, let the last MMAs finish before TMEM is released.
         if (lane == 0 && *abort_flag && last_acc >= 0)
             mbar_wait_bounded(&tfull[last_acc], last_aph, a.wait_limit, nullptr);
@@ -276,83 +338,103 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int quarter = warp & 3;   // TMEM lanes this warp may access
         const int half = ew >> 2;       // column half of the tile
         const int row_in = quarter * 32 + lane;
-        const float qnan = __int_as_float(0x7fc00000);
+        float* stage = stage_all + ew * kStageFloats;
         int it = 0;
-        for (long long t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
-            const TileCoord tc = decode_tile(t, a);
-            if (!tc.active) continue;
-            const int acc = it & 1;
-            const uint32_t aph = (uint32_t)(it >> 1) & 1u;
-            if (!warp_wait(&tfull[acc], aph)) {
-                if (lane == 0) fail();
-                break;
-            }
-            tc_fence_after();
-            const int q = tc.rb * kBM + row_in;
+        bool ok = true;
+        for (int u = blockIdx.x; u < a.nunits && ok; u += gridDim.x) {
+            const Unit un = decode_unit(u, a);
+            const int q = un.rb * kBM + row_in;
             const bool vrow = q < a.nq;
             const int p = a.q_start + q;
-            const long long grow = (long long)q * a.hkv + tc.h;
-            const int col0 = tc.c * kBN + half * 128;
-            const uint32_t taddr = tbase + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * kBN + half * 128);
-            if (MODE == kModeSample) {
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t v[32];
-                    tmem_ld32(taddr + ch * 32, v);
-                    tmem_wait(v);
-                    if (vrow) {
-                        float* dst = a.samp + grow * a.ld_samp + col0 + ch * 32;
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const int c0 = col0 + ch * 32 + j;
-                            float4 f;
-                            f.x = (long long)(c0 + 0) * a.S <= p ? __uint_as_float(v[j + 0]) : qnan;
-                            f.y = (long long)(c0 + 1) * a.S <= p ? __uint_as_float(v[j + 1]) : qnan;
-                            f.z = (long long)(c0 + 2) * a.S <= p ? __uint_as_float(v[j + 2]) : qnan;
-                            f.w = (long long)(c0 + 3) * a.S <= p ? __uint_as_float(v[j + 3]) : qnan;
-                            *reinterpret_cast<float4*>(dst + j) = f;
-                        }
-                    }
+            const long long grow = (long long)q * a.hkv + un.h;
+            // filter mode: this thread's writer slot and list region
+            const int slot = half * a.nseg + un.seg;
+            const bool down = (slot & 1) != 0;
+            uint2* region = a.cand + grow * a.ld_cand + (long long)(slot >> 1) * a.cap_pair;
+            float thr_f = 0.f;
+            if (MODE == kModeFilter) thr_f = vrow ? key_floor(__ldg(&a.thr[grow])) : __int_as_float(0x7f800000);
+            unsigned n = 0;
+            for (int c = un.c0; c < un.c1; ++c) {
+                const int acc = it & 1;
+                const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+                if (!warp_wait(&tfull[acc], aph)) {
+                    ok = false;
+                    break;
                 }
-            } else {
-                const uint32_t thr = vrow ? __ldg(&a.thr[grow]) : 0xFFFFFFFFu;
-                int n = 0;
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t v[32];
-                    tmem_ld32(taddr + ch * 32, v);
-                    tmem_wait(v);
+                tc_fence_after();
+                const int col0 = c * kBN + half * 128;
+                const uint32_t taddr = tbase + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * kBN + half * 128);
+                for (int ch = 0; ch < 4; ch += 2) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(taddr + ch * 32, v0);
+                    tmem_ld32(taddr + ch * 32 + 32, v1);
+                    tmem_wait(v0);
+                    tmem_wait(v1);
+                    if (MODE == kModeSample) {
+                        if (vrow) {
+                            uint4* dst = reinterpret_cast<uint4*>(a.samp + grow * a.ld_samp + col0 + ch * 32);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int tpos = col0 + ch * 32 + j;
-                        n += (tpos <= p && score_key(__uint_as_float(v[j])) >= thr) ? 1 : 0;
-                    }
-                }
-                unsigned w = 0;
-                if (n) w = atomicAdd(&a.cnt[grow], (unsigned)n);
-                if (__any_sync(0xffffffffu, n != 0)) {
-                    uint2* dst = a.cand + grow * a.cap;
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t v[32];
-                        tmem_ld32(taddr + ch * 32, v);
-                        tmem_wait(v);
-                        if (n) {
+                            for (int g = 0; g < 8; ++g) {
+                                uint32_t w[4];
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                const int tpos = col0 + ch * 32 + j;
-                                const uint32_t key = score_key(__uint_as_float(v[j]));
-                                if (tpos <= p && key >= thr) {
-                                    if (w < (unsigned)a.cap) dst[w] = make_uint2(key, (uint32_t)tpos);
-                                    ++w;
+                                for (int e = 0; e < 4; ++e) {
+                                    const int j = g * 8 + e * 2;
+                                    const uint32_t* src = j < 32 ? v0 : v1;
+                                    const int jj = j & 31;
+                                    const long long t0 = (long long)(col0 + ch * 32 + j) * a.S;
+                                    const uint32_t k0 = t0 <= p ? score_key(__uint_as_float(src[jj])) >> 16 : 0u;
+                                    const uint32_t k1 =
+                                        t0 + a.S <= p ? score_key(__uint_as_float(src[jj + 1])) >> 16 : 0u;
+                                    w[e] = k0 | (k1 << 16);
                                 }
+                                dst[g] = make_uint4(w[0], w[1], w[2], w[3]);
+                            }
+                        }
+                    } else {
+                        // Pass masks first (branch-free), then only the passing
+                        // entries, read back from a per-warp staging tile.
+                        const bool diag = (long long)(c + 1) * kBN - 1 > un.pmin;
+#pragma unroll
+                        for (int k = 0; k < 2; ++k) {
+                            const uint32_t* v = k ? v1 : v0;
+                            const int cb = col0 + ch * 32 + k * 32;   // first column of this chunk
+                            uint32_t m = 0;
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) m |= (__uint_as_float(v[j]) >= thr_f ? 1u : 0u) << j;
+                            if (diag) {
+                                const int lim = p - cb;   // columns cb + j with j <= lim are causal
+                                m &= lim >= 31 ? 0xFFFFFFFFu : (lim < 0 ? 0u : (2u << lim) - 1u);
+                            }
+                            if (!vrow) m = 0;
+                            if (__any_sync(0xffffffffu, m != 0u)) {
+                                float4* st4 = reinterpret_cast<float4*>(stage + lane * kStageRow);
+#pragma unroll
+                                for (int g = 0; g < 8; ++g)
+                                    st4[g] = make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
+                                                         __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
+                                __syncwarp();
+                                while (m) {
+                                    const int j = __ffs(m) - 1;
+                                    m &= m - 1u;
+                                    if (n < (unsigned)a.cap_pair) {
+                                        const unsigned at = down ? (unsigned)a.cap_pair - 1u - n : n;
+                                        region[at] = make_uint2(score_key(stage[lane * kStageRow + j]), (uint32_t)(cb + j));
+                                    }
+                                    ++n;
+                                }
+                                __syncwarp();
                             }
                         }
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+                ++it;
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
-            ++it;
+            if (MODE == kModeFilter && ok && vrow) a.cnt[grow * kMaxSlots + slot] = n;
         }
+        if (!ok && lane == 0) fail();
     }
     __syncthreads();
     if (warp == 1) {
@@ -384,21 +466,27 @@ __global__ void prefill_qbar_kernel(const uint16_t* __restrict__ qt, uint16_t* _
 
 // ---------------------------------------------------------------- selection
 struct SelArgs {
-    int hkv, nq, nq_pad, q_start, B, cap, r, S, kth;
-    long long ld_samp;
-    const float* samp;
+    int hkv, nq, nq_pad, q_start, B, cap, cap_pair, nseg, r, S, kth;
+    long long rows, ld_samp, ld_cand;
+    const uint16_t* samp;
     uint32_t* thr;
-    unsigned* cnt;
+    const unsigned* cnt;
     const uint2* cand;
     const uint16_t* qb;
     const uint16_t* kt;
     int32_t* idx;
 };
 
+constexpr int kEqList = 1024;         // boundary ties resolved by direct ranking up to this many
+
 struct SelShared {
     uint32_t hist[2048];
     int wtot[32];
     int bin, above, eqc;
+    int start[8], pre[9];
+    int fb, neq;
+    uint32_t pos_thr;
+    uint32_t eqpos[kEqList];
 };
 
 // Exclusive block-wide prefix sum of v (thread order); *total = the sum.
@@ -492,32 +580,83 @@ __device__ void block_select(F key_of, int count, int need, SelShared& sh, uint3
     *n_eq = eqc;
 }
 
-// theta_row = the kth-largest sampled score of the row (rows short enough to
-// keep every key get the smallest key, 1); also zeroes the row's count.
-__global__ void __launch_bounds__(kSelThreads) prefill_threshold_kernel(const SelArgs a) {
-    __shared__ SelShared sh;
-    __shared__ uint32_t skeys[kMaxSamples];
-    const int row = blockIdx.x;
-    const int q = row / a.hkv;
+// In a 256-bin histogram, the bin b holding the rem-th largest entry, and the
+// entries in bins above it (warp-wide; every lane gets the results).
+__device__ __forceinline__ void warp_find_bin(const uint32_t* h, int rem, int lane, int* bin, int* above, int* total) {
+    const int top = 255 - lane * 8;
+    int s = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s += (int)h[top - j];
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    *total = __shfl_sync(0xffffffffu, incl, 31);
+    const int excl = incl - s;
+    int b = -1, ab = 0;
+    if (excl < rem && rem <= incl) {
+        int c = excl;
+        for (int j = 0; j < 8; ++j) {
+            const int hb = (int)h[top - j];
+            if (c + hb >= rem) {
+                b = top - j;
+                ab = c;
+                break;
+            }
+            c += hb;
+        }
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, b >= 0);
+    const int src = m ? __ffs(m) - 1 : 0;
+    *bin = __shfl_sync(0xffffffffu, b, src);
+    *above = __shfl_sync(0xffffffffu, ab, src);
+}
+
+// theta_row (one warp per row) = the kth-largest 16-bit sampled key of the
+// row, widened to 32 bits (so at least kth sampled keys are >= theta_row);
+// rows short enough to keep every key, or with fewer than kth samples, get
+// the smallest key, 1.
+constexpr int kThrWarps = 8;
+__global__ void __launch_bounds__(kThrWarps * 32) prefill_threshold_kernel(const SelArgs a) {
+    __shared__ uint32_t hist[kThrWarps][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * kThrWarps + warp;
+    if (row >= a.rows) return;
+    const int q = (int)(row / a.hkv);
     const int p = a.q_start + q;
     if (p + 1 <= a.cap || a.samp == nullptr) {
-        if (threadIdx.x == 0) {
-            a.thr[row] = 1u;
-            a.cnt[row] = 0u;
-        }
+        if (lane == 0) a.thr[row] = 1u;
         return;
     }
     const int ms = (int)min((long long)(p / a.S + 1), a.ld_samp);
-    const float* src = a.samp + (long long)row * a.ld_samp;
-    for (int i = threadIdx.x; i < ms; i += kSelThreads) skeys[i] = score_key(__ldcg(src + i));
-    __syncthreads();
-    uint32_t theta;
-    int gt, eq, total;
-    block_select<kSelThreads>([&](int i) { return skeys[i]; }, ms, a.kth, sh, &theta, &gt, &eq, &total);
-    if (threadIdx.x == 0) {
-        a.thr[row] = total >= a.kth ? theta : 1u;
-        a.cnt[row] = 0u;
+    const uint16_t* src = a.samp + row * a.ld_samp;
+    uint32_t* h = hist[warp];
+    for (int i = lane; i < 256; i += 32) h[i] = 0u;
+    __syncwarp();
+    for (int i = lane; i < ms; i += 32) {
+        const uint32_t k = src[i];
+        if (k) atomicAdd(&h[k >> 8], 1u);
     }
+    __syncwarp();
+    int b1, ab1, total;
+    warp_find_bin(h, a.kth, lane, &b1, &ab1, &total);
+    if (total < a.kth) {
+        if (lane == 0) a.thr[row] = 1u;
+        return;
+    }
+    __syncwarp();
+    for (int i = lane; i < 256; i += 32) h[i] = 0u;
+    __syncwarp();
+    for (int i = lane; i < ms; i += 32) {
+        const uint32_t k = src[i];
+        if ((k >> 8) == (uint32_t)b1) atomicAdd(&h[k & 255u], 1u);
+    }
+    __syncwarp();
+    int b2, ab2, t2;
+    warp_find_bin(h, a.kth - ab1, lane, &b2, &ab2, &t2);
+    if (lane == 0) a.thr[row] = ((uint32_t)b1 << 24) | ((uint32_t)b2 << 16);
 }
 
 // Exact top-B of one row (dynamic shared memory: a bitmap of the row's
@@ -531,9 +670,28 @@ __global__ void __launch_bounds__(kSelThreads) prefill_select_kernel(const SelAr
     const int p = a.q_start + q;
     const int n = p + 1;
     const int need = min(a.B, n);
-    const unsigned count = __ldcg(&a.cnt[row]);
-    const bool fb = count > (unsigned)a.cap || count < (unsigned)need;
-    const uint2* cand = a.cand + (long long)row * a.cap;
+    const int slots = 2 * a.nseg;
+    const uint2* cand = a.cand + (long long)row * a.ld_cand;
+    if (threadIdx.x == 0) {
+        int tot = 0;
+        bool over = false;
+        for (int j = 0; j < slots; ++j) {
+            const unsigned c = __ldcg(&a.cnt[(long long)row * kMaxSlots + j]);
+            if (j & 1) {
+                const unsigned f = __ldcg(&a.cnt[(long long)row * kMaxSlots + j - 1]);
+                if (f + c > (unsigned)a.cap_pair) over = true;
+            }
+            const int cl = (int)min(c, (unsigned)a.cap_pair);
+            sh.start[j] = (j >> 1) * a.cap_pair + ((j & 1) ? a.cap_pair - cl : 0);
+            sh.pre[j] = tot;
+            tot += cl;
+        }
+        sh.pre[slots] = tot;
+        sh.fb = (over || tot < need) ? 1 : 0;
+        sh.neq = 0;
+    }
+    __syncthreads();
+    const bool fb = sh.fb != 0;
     const int r = a.r;
     if (fb) {
         for (int c = threadIdx.x; c < r; c += kSelThreads)
@@ -556,30 +714,70 @@ __global__ void __launch_bounds__(kSelThreads) prefill_select_kernel(const SelAr
         }
         return score_key(acc);
     };
-    auto key_of = [&](int i) -> uint32_t { return fb ? recompute(i) : __ldcg(&cand[i]).x; };
-    auto pos_of = [&](int i) -> uint32_t { return fb ? (uint32_t)i : __ldcg(&cand[i]).y; };
-    const int items = fb ? n : (int)count;
+    auto entry = [&](int i) -> uint2 {
+        int j = 0;
+        while (j + 1 < slots && i >= sh.pre[j + 1]) ++j;
+        return __ldcg(&cand[sh.start[j] + (i - sh.pre[j])]);
+    };
+    auto key_of = [&](int i) -> uint32_t { return fb ? recompute(i) : entry(i).x; };
+    const int items = fb ? n : sh.pre[slots];
 
     uint32_t theta;
     int gt, eq, total;
     block_select<kSelThreads>(key_of, items, need, sh, &theta, &gt, &eq, &total);
     uint32_t pos_thr = 0xFFFFFFFFu;
-    if (theta != 0u && eq > need - gt) {
-        // Equal keys at the boundary: keep the need - gt lowest positions.
-        uint32_t th2;
-        int g2, e2, t2;
-        block_select<kSelThreads>(
-            [&](int i) -> uint32_t { return key_of(i) == theta ? ~pos_of(i) : 0u; }, items, need - gt, sh, &th2, &g2,
-            &e2, &t2);
-        pos_thr = ~th2;
+    const int need_eq = need - gt;
+    if (theta != 0u && eq > need_eq) {
+        // Equal keys at the boundary: keep the need_eq lowest positions.
+        if (eq <= kEqList) {
+            for (int i = threadIdx.x; i < items; i += kSelThreads) {
+                uint32_t k, pos;
+                if (fb) {
+                    k = recompute(i);
+                    pos = (uint32_t)i;
+                } else {
+                    const uint2 e = entry(i);
+                    k = e.x;
+                    pos = e.y;
+                }
+                if (k == theta) sh.eqpos[atomicAdd(&sh.neq, 1)] = pos;
+            }
+            __syncthreads();
+            for (int i = threadIdx.x; i < eq; i += kSelThreads) {
+                const uint32_t mine = sh.eqpos[i];
+                int rank = 0;
+                for (int j = 0; j < eq; ++j) rank += sh.eqpos[j] < mine ? 1 : 0;
+                if (rank == need_eq - 1) sh.pos_thr = mine;
+            }
+            __syncthreads();
+            pos_thr = sh.pos_thr;
+        } else {
+            uint32_t th2;
+            int g2, e2, t2;
+            block_select<kSelThreads>(
+                [&](int i) -> uint32_t {
+                    if (fb) return recompute(i) == theta ? ~(uint32_t)i : 0u;
+                    const uint2 e = entry(i);
+                    return e.x == theta ? ~e.y : 0u;
+                },
+                items, need_eq, sh, &th2, &g2, &e2, &t2);
+            pos_thr = ~th2;
+        }
     }
     const int nw = (n + 31) >> 5;
     for (int w = threadIdx.x; w < nw; w += kSelThreads) bitmap[w] = 0u;
     __syncthreads();
     for (int i = threadIdx.x; i < items; i += kSelThreads) {
-        const uint32_t k = key_of(i);
+        uint32_t k, pos;
+        if (fb) {
+            k = recompute(i);
+            pos = (uint32_t)i;
+        } else {
+            const uint2 e = entry(i);
+            k = e.x;
+            pos = e.y;
+        }
         if (k == 0u) continue;
-        const uint32_t pos = pos_of(i);
         if (k > theta || (k == theta && pos <= pos_thr)) atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
     }
     __syncthreads();
@@ -653,29 +851,39 @@ PrefillPlan plan_prefill(int hq, int hkv, int r, int T, int nq, int B) {
     const long long expect = (long long)P.kth * S;               // keys expected above theta
     long long cap = 2 * expect;
     if (cap < B + B / 2 + 512) cap = B + B / 2 + 512;
+    if (cap < 2048) cap = 2048;
     P.cap = (int)((cap + 255) / 256 * 256);
     P.sample = T > P.cap;
     const long long m = ((long long)T + S - 1) / S;
     P.ncol_sample = (int)((m + kBN - 1) / kBN);
     P.ld_samp = (long long)P.ncol_sample * kBN;
-    const size_t st = (size_t)(kBM + kBN) * r * 2;
-    int stages = (int)((192 * 1024) / st);
+    const size_t a_bytes = (size_t)kBM * r * 2, b_bytes = (size_t)kBN * r * 2;
+    const size_t staging = (size_t)kEpiWarps * kStageFloats * 4;
+    const size_t fixed = (2 * kMaxStages + 8) * 8 + 16 + 1024;   // barriers, TMEM slot, alignment slack
+    const size_t budget = 227 * 1024 - fixed - staging;
+    int a_slots = 2;
+    long long stages = ((long long)budget - 2 * (long long)a_bytes) / (long long)b_bytes;
+    if (stages < 3) {
+        a_slots = 1;
+        stages = ((long long)budget - (long long)a_bytes) / (long long)b_bytes;
+    }
     if (stages > kMaxStages) stages = kMaxStages;
-    P.stages = stages;
-    size_t smem = stages * st + 2 * kMaxStages * 8 + 4 * 8 + 16 + 1024;
+    P.stages = (int)stages;
+    P.a_slots = a_slots;
+    size_t smem = a_slots * a_bytes + P.stages * b_bytes + staging + fixed;
     if (smem < 120 * 1024) smem = 120 * 1024;   // one CTA per SM: each holds all 512 TMEM columns
     P.gemm_smem = (int)smem;
     size_t off = 0;
     P.off_qb = off;
     off = align256(off + (size_t)hkv * P.nq_pad * r * 2);
     P.off_samp = off;
-    if (P.sample) off = align256(off + (size_t)P.rows * P.ld_samp * 4);
+    if (P.sample) off = align256(off + (size_t)P.rows * P.ld_samp * 2);
     P.off_thr = off;
     off = align256(off + (size_t)P.rows * 4);
     P.off_cnt = off;
-    off = align256(off + (size_t)P.rows * 4);
+    off = align256(off + (size_t)P.rows * kMaxSlots * 4);
     P.off_cand = off;
-    off = align256(off + (size_t)P.rows * P.cap * 8);
+    off = align256(off + (size_t)P.rows * 2 * P.cap * 8);   // room for the 4-segment layout
     P.bytes = off;
     return P;
 }
@@ -684,10 +892,11 @@ cudaError_t launch_prefill_index(const LaunchCtx& ctx, const PrefillPlan& P, con
                                  int hq, int hkv, int r, int T, int nq, int q_start, int B, int32_t* idx, uint8_t* ws,
                                  unsigned* status) {
     uint16_t* qb = reinterpret_cast<uint16_t*>(ws + P.off_qb);
-    float* samp = P.sample ? reinterpret_cast<float*>(ws + P.off_samp) : nullptr;
+    uint16_t* samp = P.sample ? reinterpret_cast<uint16_t*>(ws + P.off_samp) : nullptr;
     uint32_t* thr = reinterpret_cast<uint32_t*>(ws + P.off_thr);
     unsigned* cnt = reinterpret_cast<unsigned*>(ws + P.off_cnt);
     uint2* cand = reinterpret_cast<uint2*>(ws + P.off_cand);
+    const long long pmax = (long long)q_start + nq - 1;
 
     {
         const long long total = (long long)hkv * P.nq_pad * r;
@@ -699,7 +908,8 @@ cudaError_t launch_prefill_index(const LaunchCtx& ctx, const PrefillPlan& P, con
         !make_map(&mB, kt, (uint64_t)hkv * r, (uint64_t)T, (uint64_t)hkv * r * 2, box_in, kBN))
         return cudaErrorInvalidValue;
     const long long nsamp_rows = ((long long)T + P.S - 1) / P.S;
-    if (P.sample &&
+    const bool any_sample = P.sample && pmax + 1 > P.cap;
+    if (any_sample &&
         !make_map(&mS, kt, (uint64_t)hkv * r, (uint64_t)nsamp_rows, (uint64_t)hkv * r * 2 * P.S, box_in, kBN))
         return cudaErrorInvalidValue;
 
@@ -709,15 +919,20 @@ cudaError_t launch_prefill_index(const LaunchCtx& ctx, const PrefillPlan& P, con
     g.nq = nq;
     g.nq_pad = P.nq_pad;
     g.q_start = q_start;
-    g.rb_per_head = P.nq_pad / kBM;
+    g.nrb = P.nq_pad / kBM;
     g.stages = P.stages;
+    g.a_slots = P.a_slots;
     g.thr = thr;
     g.cnt = cnt;
     g.cand = cand;
-    g.cap = P.cap;
     g.status = status;
     g.wait_limit = ctx.wait_limit;
-    const long long pmax = (long long)q_start + nq - 1;
+
+    // Filter pass layout: 4 column segments per row block when rows span many
+    // tiles (enough units to fill the GPU), else 2 or 1.
+    const int ncol_f = (int)((pmax + 1 + kBN - 1) / kBN);
+    const int nseg = ncol_f >= 16 ? 4 : (ncol_f >= 2 ? 2 : 1);
+    const int cap_pair = nseg == 1 ? P.cap : P.cap / 2;
 
     SelArgs s{};
     s.hkv = hkv;
@@ -726,41 +941,46 @@ cudaError_t launch_prefill_index(const LaunchCtx& ctx, const PrefillPlan& P, con
     s.q_start = q_start;
     s.B = B;
     s.cap = P.cap;
+    s.cap_pair = cap_pair;
+    s.nseg = nseg;
     s.r = r;
     s.S = P.S;
     s.kth = P.kth;
+    s.rows = P.rows;
     s.ld_samp = P.ld_samp;
-    s.samp = samp;
+    s.ld_cand = (long long)nseg * cap_pair;
+    s.samp = any_sample ? samp : nullptr;
     s.thr = thr;
     s.cnt = cnt;
     s.cand = cand;
     s.qb = qb;
     s.kt = kt;
     s.idx = idx;
-    const bool any_sample = P.sample && pmax + 1 > P.cap;
 
     cudaError_t e;
     if (any_sample) {
         GemmArgs gs = g;
         gs.S = P.S;
-        gs.ncol_tiles = (int)((pmax / P.S + 1 + kBN - 1) / kBN);
-        gs.ntiles = (long long)hkv * gs.ncol_tiles * gs.rb_per_head;
+        gs.ncol = (int)((pmax / P.S + 1 + kBN - 1) / kBN);
+        gs.nseg = 1;
+        gs.nunits = hkv * gs.nrb;
         gs.samp = samp;
         gs.ld_samp = P.ld_samp;
         if ((e = ensure_dyn_smem((const void*)prefill_gemm_kernel<kModeSample>, P.gemm_smem)) != cudaSuccess) return e;
-        const unsigned grid = (unsigned)(gs.ntiles < ctx.num_sms ? gs.ntiles : ctx.num_sms);
+        const unsigned grid = (unsigned)(gs.nunits < ctx.num_sms ? gs.nunits : ctx.num_sms);
         prefill_gemm_kernel<kModeSample><<<grid, kGemmThreads, P.gemm_smem, ctx.stream>>>(mA, mS, gs);
-    } else {
-        s.samp = nullptr;
     }
-    prefill_threshold_kernel<<<(unsigned)P.rows, kSelThreads, 0, ctx.stream>>>(s);
+    prefill_threshold_kernel<<<(unsigned)((P.rows + kThrWarps - 1) / kThrWarps), kThrWarps * 32, 0, ctx.stream>>>(s);
     {
         GemmArgs gf = g;
         gf.S = 1;
-        gf.ncol_tiles = (int)((pmax + 1 + kBN - 1) / kBN);
-        gf.ntiles = (long long)hkv * gf.ncol_tiles * gf.rb_per_head;
+        gf.ncol = ncol_f;
+        gf.nseg = nseg;
+        gf.nunits = hkv * nseg * gf.nrb;
+        gf.cap_pair = cap_pair;
+        gf.ld_cand = (long long)nseg * cap_pair;
         if ((e = ensure_dyn_smem((const void*)prefill_gemm_kernel<kModeFilter>, P.gemm_smem)) != cudaSuccess) return e;
-        const unsigned grid = (unsigned)(gf.ntiles < ctx.num_sms ? gf.ntiles : ctx.num_sms);
+        const unsigned grid = (unsigned)(gf.nunits < ctx.num_sms ? gf.nunits : ctx.num_sms);
         prefill_gemm_kernel<kModeFilter><<<grid, kGemmThreads, P.gemm_smem, ctx.stream>>>(mA, mB, gf);
     }
     {
