@@ -247,6 +247,23 @@ def run_reference(args, rank, world):
         return 0
     from indexed_sparse_attention_kv_b200 import inputs as I
 
+    if args.workload == "prefill_128k":
+        w = I.workload("prefill_128k")
+        x = I.make_prefill_inputs(w)
+        cpu_prefill_sample(w, x, budget_s=0.0, max_rows=max(1, args.warmup))
+        v, n, el = cpu_prefill_sample(w, x, budget_s=0.0, max_rows=max(1, args.steps))
+        line = {
+            "impl": "reference", "metric": PREFILL_METRIC, "value": v, "unit": PREFILL_UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "nq": w.nq, "T": w.T, "hq": w.hq, "hkv": w.hkv, "d": w.d, "r": w.r,
+                       "B": w.B},
+            "cpu_baseline": {"value": v, "unit": PREFILL_UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{n} query rows of 4096 per timed run, scaled to whole prefills"},
+            "e2e": {"value": v, "unit": PREFILL_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return 0
     w = I.workload(WORKLOAD)
     x = I.make_decode_inputs(w)
     cores = blas_threads()
@@ -417,7 +434,7 @@ def run_ours(args, rank, world, local_rank):
             "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_dict(w, {"parallelism": f"replicas{world}" if world > 1 else "single"}),
-            "roofline": {"bound": "hbm", "kernel": "score_flat_kernel", "achieved": achieved, "peak": peak,
+            "roofline": {"bound": "hbm", "kernel": "score_q64_kernel (lsa_score)", "achieved": achieved, "peak": peak,
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_kind": peak_kind, "algorithmic_bytes_per_launch": scorer_bytes,
                          "avg_launch_ms": score_ms},
@@ -429,6 +446,167 @@ def run_ours(args, rank, world, local_rank):
                     "h2d_bytes_per_step": hq.numel() * 2 + hqt.numel() * 2,
                     "d2h_bytes_per_step": hout.numel() * 2 + hidx.numel() * 4},
             "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "clocks": clocks,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+PREFILL_METRIC = "prefill steps/s at 128K (4096 causal queries, B=2048): indexer + indexed attention"
+PREFILL_UNIT = "prefills/s"
+PREFILL_KERNELS = 6       # group mean, sampled GEMM, thresholds, filter GEMM, selection, attention
+
+
+def prefill_scoring_flop(w):
+    """Useful scoring FLOPs of one prefill: 2 r per causal (query, key, KV head)."""
+    q0 = w.T - w.nq
+    pairs = sum(q0 + i + 1 for i in range(w.nq)) * w.hkv
+    return 2 * pairs * w.r
+
+
+def measured_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def cpu_prefill_sample(w, x, budget_s=12.0, max_rows=None):
+    """Oracle prefill (index + attention) on query rows until about budget_s
+    seconds; returns (prefills/s, rows, seconds)."""
+    import torch
+
+    import oracle.lsa_oracle as O
+
+    q0 = int(x["q_start"])
+    kt = x["kt"].to(torch.float32).numpy()
+    done, elapsed = 0, 0.0
+    while True:
+        i = (done * 577) % w.nq
+        qt = x["qt"][i:i + 1].to(torch.float32).numpy()
+        q = x["q"][i].to(torch.float32).numpy()
+        ts = time.perf_counter()
+        idx = O.prefill_index(qt, [q0 + i], kt, w.B)[0]
+        sel = [idx[h][idx[h] >= 0] for h in range(w.hkv)]
+        for h in range(w.hkv):
+            k_rows = x["k"][sel[h], h:h + 1].to(torch.float32).numpy()
+            v_rows = x["v"][sel[h], h:h + 1].to(torch.float32).numpy()
+            import numpy as np
+            O.indexed_attention(q[h * w.G:(h + 1) * w.G], k_rows, v_rows, np.arange(len(sel[h]))[None], w.scale)
+        elapsed += time.perf_counter() - ts
+        done += 1
+        if elapsed >= budget_s or (max_rows and done >= max_rows):
+            break
+    return done / w.nq / elapsed, done, elapsed
+
+
+def run_prefill(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import indexed_sparse_attention_kv_b200 as lsa
+    from indexed_sparse_attention_kv_b200 import inputs as I
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    lsa.lib()
+    w = I.workload("prefill_128k")
+    x = I.make_prefill_inputs(w, seed=rank_seed(w, rank))
+    q0 = int(x["q_start"])
+    d = {k: x[k].to(dev) for k in ("q", "qt", "k", "v", "kt")}
+    dims = lsa.lsa_dims(1, w.hq, w.hkv, w.d, w.r, w.T)
+    ws = lsa.prefill_workspace(dims, w.nq, w.B, device=dev)
+    idx = torch.empty((w.nq, w.hkv, w.B), dtype=torch.int32, device=dev)
+    out = torch.empty_like(d["q"])
+    stream = torch.cuda.current_stream(dev)
+
+    def index():
+        lsa.lsa_prefill_index(d["qt"], d["kt"], q0, w.B, idx=idx, ws=ws)
+
+    def attn():
+        lsa.lsa_prefill_attn(d["q"], d["k"], d["v"], idx, out=out, ws=ws)
+
+    def step():
+        index()
+        attn()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    status = lsa.lsa_read_device_status(ws)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = e0.elapsed_time(e1)
+    clocks = clk.summary()
+    comp = {}
+    for name, fn in (("indexer", index), ("attention", attn)):
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        comp[name] = e0.elapsed_time(e1) / args.steps
+    # end to end: H2D of the step's queries, D2H of index sets and outputs
+    hq, hqt = x["q"].pin_memory(), x["qt"].pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hidx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        d["q"].copy_(hq, non_blocking=True)
+        d["qt"].copy_(hqt, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+        hidx.copy_(idx, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = e0.elapsed_time(e1)
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
+    if rank == 0:
+        peak, peak_kind = measured_tflops()
+        flop = prefill_scoring_flop(w)
+        achieved = flop / (comp["indexer"] / 1e3) / 1e12
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            v, n, el = cpu_prefill_sample(w, x, budget_s=args.cpu_budget)
+            cpu = {"value": v, "unit": PREFILL_UNIT, "cores": blas_threads(), "kind": "oracle",
+                   "sample": f"{n} query rows of 4096 ({el:.1f} s), scaled to whole prefills"}
+        line = {
+            "metric": PREFILL_METRIC, "value": weak_value(world, args.steps, ms), "unit": PREFILL_UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "nq": w.nq, "q_start": q0, "T": w.T, "hq": w.hq, "hkv": w.hkv,
+                       "d": w.d, "r": w.r, "B": w.B,
+                       "l2": "inputs exceed L2 (128 MiB projected keys, 512 MiB K/V)"},
+            "roofline": {"bound": "tensor", "kernel": "lsa_prefill_index (score GEMMs + selection)",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "traffic": None, "peak_kind": peak_kind, "algorithmic_flop_per_launch": flop,
+                         "avg_launch_ms": comp["indexer"]},
+            "components_ms": comp,
+            "cpu_baseline": cpu,
+            "e2e": {"value": weak_value(world, args.steps, ms_e2e), "unit": PREFILL_UNIT,
+                    "h2d_bytes_per_step": hq.numel() * 2 + hqt.numel() * 2,
+                    "d2h_bytes_per_step": hout.numel() * 2 + hidx.numel() * 4},
+            "gpu_launches": PREFILL_KERNELS * args.steps,
             "clocks": clocks,
             "device_status": status,
         }
@@ -476,6 +654,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["decode_128k", "prefill_128k"], default="decode_128k",
+                    help="decode_128k (the headline) or prefill_128k (indexer + indexed attention)")
     ap.add_argument("--ncu-case", choices=["score", "topk", "attn", "step"], default=None,
                     help="run one component on a reduced 128K case (batch 2) for an ncu capture; no JSON")
     args = ap.parse_args(argv)
@@ -496,6 +676,8 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.workload == "prefill_128k":
+            return run_prefill(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
