@@ -111,7 +111,9 @@ struct AttnLayout {
     static constexpr int kMerge = (kAttnWarps - 1) * (G * D + 2 * 16) * 4;   // warps 1..3: O, m, l
     static constexpr int kRows = 4 * kNT * 4;                      // row-id ring (>= stages + 1)
     static constexpr int kFixed = kMerge + kRows;
-    static constexpr int kStages = (227 * 1024 / 2 - kFixed) / kStage >= 3 ? 3 : 2;
+    // two stages: three CTAs (12 warps) fit per SM, which hides the fixed
+    // latencies of the per-warp MMA / softmax chain better than a third stage
+    static constexpr int kStages = 2;
     static constexpr int kTotal = kStages * kStage + kFixed;
 };
 

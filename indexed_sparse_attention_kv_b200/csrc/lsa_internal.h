@@ -1,6 +1,7 @@
 // Internal launchers shared by the kernel files and the C-ABI layer.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -46,6 +47,13 @@ inline cudaError_t cached_occupancy(const void* kern, int threads, size_t smem, 
     if (e == cudaSuccess) done[key] = *occ;
     return e;
 }
+
+// 2-D bf16 tensor map over `outer` rows of `inner` elements, rows `row_bytes`
+// apart, boxes of box_inner x box_outer, swizzled to the box row width (32,
+// 64 or 128 bytes). Returns false if the driver entry point or the encoding
+// fails.
+bool make_tensor_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                        uint32_t box_inner, uint32_t box_outer);
 
 struct LaunchCtx {
     cudaStream_t stream;

@@ -518,12 +518,12 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wtot, int* total) {
 }
 
 // Block-wide radix selection (11 + 11 + 10 bits) of the need-th largest
-// non-zero key among key_of(i), i in [0, count). Results, identical in every
-// thread: *theta = that key, *n_gt = keys above it, *n_eq = keys equal to it,
-// *total = non-zero keys. With fewer than `need` keys: theta = 0, n_gt = total.
-template <int NT, class F>
-__device__ void block_select(F key_of, int count, int need, SelShared& sh, uint32_t* theta, int* n_gt, int* n_eq,
-                             int* total) {
+// non-zero key. `visit(f)` calls f(key, position) for every item this thread
+// holds (key 0 = no item). Results, identical in every thread: *theta = that
+// key, *n_gt = keys above it, *n_eq = keys equal to it, *total = non-zero
+// keys. With fewer than `need` keys: theta = 0, n_gt = total.
+template <int NT, class V>
+__device__ void block_select(V visit, int need, SelShared& sh, uint32_t* theta, int* n_gt, int* n_eq, int* total) {
     const int tid = threadIdx.x;
     uint32_t prefix = 0, pmask = 0;
     int rem = need, gt = 0, eqc = 0;
@@ -532,10 +532,9 @@ __device__ void block_select(F key_of, int count, int need, SelShared& sh, uint3
         const int nb = pass == 2 ? 1024 : 2048;
         for (int i = tid; i < 2048; i += NT) sh.hist[i] = 0;
         __syncthreads();
-        for (int i = tid; i < count; i += NT) {
-            const uint32_t k = key_of(i);
+        visit([&](uint32_t k, uint32_t) {
             if (k != 0u && (k & pmask) == prefix) atomicAdd(&sh.hist[(k >> shift) & (uint32_t)(nb - 1)], 1u);
-        }
+        });
         __syncthreads();
         const int per = nb / NT;
         const int top = nb - 1 - tid * per;
@@ -660,88 +659,26 @@ __global__ void __launch_bounds__(kThrWarps * 32) prefill_threshold_kernel(const
 }
 
 // Exact top-B of one row (dynamic shared memory: a bitmap of the row's
-// positions, 4 * ceil((q_start + nq) / 32) bytes).
-__global__ void __launch_bounds__(kSelThreads) prefill_select_kernel(const SelArgs a) {
-    __shared__ SelShared sh;
-    __shared__ float sq[128];
-    extern __shared__ uint32_t bitmap[];
-    const int row = blockIdx.x;
-    const int q = row / a.hkv, h = row % a.hkv;
-    const int p = a.q_start + q;
-    const int n = p + 1;
-    const int need = min(a.B, n);
-    const int slots = 2 * a.nseg;
-    const uint2* cand = a.cand + (long long)row * a.ld_cand;
-    if (threadIdx.x == 0) {
-        int tot = 0;
-        bool over = false;
-        for (int j = 0; j < slots; ++j) {
-            const unsigned c = __ldcg(&a.cnt[(long long)row * kMaxSlots + j]);
-            if (j & 1) {
-                const unsigned f = __ldcg(&a.cnt[(long long)row * kMaxSlots + j - 1]);
-                if (f + c > (unsigned)a.cap_pair) over = true;
-            }
-            const int cl = (int)min(c, (unsigned)a.cap_pair);
-            sh.start[j] = (j >> 1) * a.cap_pair + ((j & 1) ? a.cap_pair - cl : 0);
-            sh.pre[j] = tot;
-            tot += cl;
-        }
-        sh.pre[slots] = tot;
-        sh.fb = (over || tot < need) ? 1 : 0;
-        sh.neq = 0;
-    }
-    __syncthreads();
-    const bool fb = sh.fb != 0;
-    const int r = a.r;
-    if (fb) {
-        for (int c = threadIdx.x; c < r; c += kSelThreads)
-            sq[c] = __uint_as_float((uint32_t)a.qb[((long long)h * a.nq_pad + q) * r + c] << 16);
-        __syncthreads();
-    }
-    // Scores recomputed on the CUDA cores (fallback rows only): fp32 FMAs over
-    // the r channels in order.
-    auto recompute = [&](int t) -> uint32_t {
-        const uint4* kr = reinterpret_cast<const uint4*>(a.kt + ((long long)t * a.hkv + h) * r);
-        float acc = 0.f;
-        for (int c8 = 0; c8 < r / 8; ++c8) {
-            const uint4 w = __ldg(kr + c8);
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                acc = fmaf(sq[c8 * 8 + 2 * j], bf16lo(ws[j]), acc);
-                acc = fmaf(sq[c8 * 8 + 2 * j + 1], bf16hi(ws[j]), acc);
-            }
-        }
-        return score_key(acc);
-    };
-    auto entry = [&](int i) -> uint2 {
-        int j = 0;
-        while (j + 1 < slots && i >= sh.pre[j + 1]) ++j;
-        return __ldcg(&cand[sh.start[j] + (i - sh.pre[j])]);
-    };
-    auto key_of = [&](int i) -> uint32_t { return fb ? recompute(i) : entry(i).x; };
-    const int items = fb ? n : sh.pre[slots];
+// positions, 4 * ceil((q_start + nq) / 32) bytes). The row's candidates are
+// loaded once into registers (kSelItems per thread); longer lists are read
+// from global memory on every pass, and rows re-done from scratch recompute
+// their scores.
+constexpr int kSelItems = 16;
 
+template <class V>
+__device__ __forceinline__ void select_and_emit(V visit, int need, int n, SelShared& sh, uint32_t* bitmap,
+                                                int32_t* out, int B) {
     uint32_t theta;
     int gt, eq, total;
-    block_select<kSelThreads>(key_of, items, need, sh, &theta, &gt, &eq, &total);
+    block_select<kSelThreads>(visit, need, sh, &theta, &gt, &eq, &total);
     uint32_t pos_thr = 0xFFFFFFFFu;
     const int need_eq = need - gt;
     if (theta != 0u && eq > need_eq) {
         // Equal keys at the boundary: keep the need_eq lowest positions.
         if (eq <= kEqList) {
-            for (int i = threadIdx.x; i < items; i += kSelThreads) {
-                uint32_t k, pos;
-                if (fb) {
-                    k = recompute(i);
-                    pos = (uint32_t)i;
-                } else {
-                    const uint2 e = entry(i);
-                    k = e.x;
-                    pos = e.y;
-                }
+            visit([&](uint32_t k, uint32_t pos) {
                 if (k == theta) sh.eqpos[atomicAdd(&sh.neq, 1)] = pos;
-            }
+            });
             __syncthreads();
             for (int i = threadIdx.x; i < eq; i += kSelThreads) {
                 const uint32_t mine = sh.eqpos[i];
@@ -755,31 +692,17 @@ __global__ void __launch_bounds__(kSelThreads) prefill_select_kernel(const SelAr
             uint32_t th2;
             int g2, e2, t2;
             block_select<kSelThreads>(
-                [&](int i) -> uint32_t {
-                    if (fb) return recompute(i) == theta ? ~(uint32_t)i : 0u;
-                    const uint2 e = entry(i);
-                    return e.x == theta ? ~e.y : 0u;
-                },
-                items, need_eq, sh, &th2, &g2, &e2, &t2);
+                [&](auto f) { visit([&](uint32_t k, uint32_t pos) { f(k == theta ? ~pos : 0u, pos); }); }, need_eq,
+                sh, &th2, &g2, &e2, &t2);
             pos_thr = ~th2;
         }
     }
     const int nw = (n + 31) >> 5;
     for (int w = threadIdx.x; w < nw; w += kSelThreads) bitmap[w] = 0u;
     __syncthreads();
-    for (int i = threadIdx.x; i < items; i += kSelThreads) {
-        uint32_t k, pos;
-        if (fb) {
-            k = recompute(i);
-            pos = (uint32_t)i;
-        } else {
-            const uint2 e = entry(i);
-            k = e.x;
-            pos = e.y;
-        }
-        if (k == 0u) continue;
-        if (k > theta || (k == theta && pos <= pos_thr)) atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
-    }
+    visit([&](uint32_t k, uint32_t pos) {
+        if (k != 0u && (k > theta || (k == theta && pos <= pos_thr))) atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
+    });
     __syncthreads();
     const int per = (nw + kSelThreads - 1) / kSelThreads;
     const int w0 = min(nw, (int)threadIdx.x * per), w1 = min(nw, w0 + per);
@@ -787,17 +710,118 @@ __global__ void __launch_bounds__(kSelThreads) prefill_select_kernel(const SelAr
     for (int w = w0; w < w1; ++w) c += __popc(bitmap[w]);
     int nsel = 0;
     int o = block_excl_scan<kSelThreads>(c, sh.wtot, &nsel);
-    int32_t* out = a.idx + (long long)row * a.B;
     for (int w = w0; w < w1; ++w) {
         uint32_t bits = bitmap[w];
         while (bits) {
             const int b = __ffs(bits) - 1;
             bits &= bits - 1u;
-            if (o < a.B) out[o] = w * 32 + b;
+            if (o < B) out[o] = w * 32 + b;
             ++o;
         }
     }
-    for (int j = nsel + threadIdx.x; j < a.B; j += kSelThreads) out[j] = -1;
+    for (int j = nsel + threadIdx.x; j < B; j += kSelThreads) out[j] = -1;
+}
+
+__global__ void __launch_bounds__(kSelThreads) prefill_select_kernel(const SelArgs a) {
+    __shared__ SelShared sh;
+    __shared__ float sq[128];
+    extern __shared__ uint32_t bitmap[];
+    const int row = blockIdx.x;
+    const int q = row / a.hkv, h = row % a.hkv;
+    const int p = a.q_start + q;
+    const int n = p + 1;
+    const int need = min(a.B, n);
+    const int slots = 2 * a.nseg;
+    const uint2* cand = a.cand + (long long)row * a.ld_cand;
+    int32_t* out = a.idx + (long long)row * a.B;
+    if (threadIdx.x < 32) {   // writer counts -> list ranges, overflow check (warp 0)
+        const int lane = threadIdx.x;
+        const unsigned c = lane < slots ? __ldcg(&a.cnt[(long long)row * kMaxSlots + lane]) : 0u;
+        const unsigned partner = __shfl_xor_sync(0xffffffffu, c, 1);
+        const bool over = (lane < slots) && (lane & 1) && c + partner > (unsigned)a.cap_pair;
+        const int cl = (int)min(c, (unsigned)a.cap_pair);
+        int incl = cl;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane < slots) {
+            sh.start[lane] = (lane >> 1) * a.cap_pair + ((lane & 1) ? a.cap_pair - cl : 0);
+            sh.pre[lane] = incl - cl;
+        }
+        const int tot = __shfl_sync(0xffffffffu, incl, 31);
+        const bool any_over = __any_sync(0xffffffffu, over);
+        if (lane == 0) {
+            sh.pre[slots] = tot;
+            sh.fb = (any_over || tot < need) ? 1 : 0;
+            sh.neq = 0;
+        }
+    }
+    __syncthreads();
+    const bool fb = sh.fb != 0;
+    const int items = sh.pre[slots];
+    auto entry = [&](int i) -> uint2 {
+        int j = 0;
+        while (j + 1 < slots && i >= sh.pre[j + 1]) ++j;
+        return __ldcg(&cand[sh.start[j] + (i - sh.pre[j])]);
+    };
+    if (!fb && items <= kSelThreads * kSelItems) {
+        uint32_t kk[kSelItems], pp[kSelItems];
+#pragma unroll
+        for (int it = 0; it < kSelItems; ++it) {
+            const int i = threadIdx.x + it * kSelThreads;
+            kk[it] = 0u;
+            pp[it] = 0u;
+            if (i < items) {
+                const uint2 e = entry(i);
+                kk[it] = e.x;
+                pp[it] = e.y;
+            }
+        }
+        select_and_emit(
+            [&](auto f) {
+#pragma unroll
+                for (int it = 0; it < kSelItems; ++it)
+                    if (kk[it]) f(kk[it], pp[it]);
+            },
+            need, n, sh, bitmap, out, a.B);
+    } else if (!fb) {
+        select_and_emit(
+            [&](auto f) {
+                for (int i = threadIdx.x; i < items; i += kSelThreads) {
+                    const uint2 e = entry(i);
+                    f(e.x, e.y);
+                }
+            },
+            need, n, sh, bitmap, out, a.B);
+    } else {
+        // Re-done from scratch: scores recomputed on the CUDA cores (fp32 FMAs
+        // over the r channels in order) for every causal position.
+        const int r = a.r;
+        for (int c = threadIdx.x; c < r; c += kSelThreads)
+            sq[c] = __uint_as_float((uint32_t)a.qb[((long long)h * a.nq_pad + q) * r + c] << 16);
+        __syncthreads();
+        auto recompute = [&](int t) -> uint32_t {
+            const uint4* kr = reinterpret_cast<const uint4*>(a.kt + ((long long)t * a.hkv + h) * r);
+            float acc = 0.f;
+            for (int c8 = 0; c8 < r / 8; ++c8) {
+                const uint4 w = __ldg(kr + c8);
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc = fmaf(sq[c8 * 8 + 2 * j], bf16lo(ws[j]), acc);
+                    acc = fmaf(sq[c8 * 8 + 2 * j + 1], bf16hi(ws[j]), acc);
+                }
+            }
+            return score_key(acc);
+        };
+        select_and_emit(
+            [&](auto f) {
+                for (int t = threadIdx.x; t < n; t += kSelThreads) f(recompute(t), (uint32_t)t);
+            },
+            need, n, sh, bitmap, out, a.B);
+    }
 }
 
 // ---------------------------------------------------------------- host side
@@ -814,9 +838,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+}  // namespace
+
 // 2-D bf16 tensor map: `outer` rows of `inner` elements, rows `row_bytes`
 // apart; boxes of box_inner x box_outer, swizzled to the box's row width.
-bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+bool make_tensor_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
               uint32_t box_inner, uint32_t box_outer) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
@@ -832,10 +860,6 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
                CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-size_t align256(size_t x) { return (x + 255) / 256 * 256; }
-
-}  // namespace
 
 PrefillPlan plan_prefill(int hq, int hkv, int r, int T, int nq, int B) {
     PrefillPlan P{};
@@ -904,13 +928,13 @@ cudaError_t launch_prefill_index(const LaunchCtx& ctx, const PrefillPlan& P, con
     }
     CUtensorMap mA, mB, mS;
     const uint32_t box_in = r < 64 ? (uint32_t)r : 64u;
-    if (!make_map(&mA, qb, (uint64_t)r, (uint64_t)hkv * P.nq_pad, (uint64_t)r * 2, box_in, kBM) ||
-        !make_map(&mB, kt, (uint64_t)hkv * r, (uint64_t)T, (uint64_t)hkv * r * 2, box_in, kBN))
+    if (!make_tensor_map_2d(&mA, qb, (uint64_t)r, (uint64_t)hkv * P.nq_pad, (uint64_t)r * 2, box_in, kBM) ||
+        !make_tensor_map_2d(&mB, kt, (uint64_t)hkv * r, (uint64_t)T, (uint64_t)hkv * r * 2, box_in, kBN))
         return cudaErrorInvalidValue;
     const long long nsamp_rows = ((long long)T + P.S - 1) / P.S;
     const bool any_sample = P.sample && pmax + 1 > P.cap;
     if (any_sample &&
-        !make_map(&mS, kt, (uint64_t)hkv * r, (uint64_t)nsamp_rows, (uint64_t)hkv * r * 2 * P.S, box_in, kBN))
+        !make_tensor_map_2d(&mS, kt, (uint64_t)hkv * r, (uint64_t)nsamp_rows, (uint64_t)hkv * r * 2 * P.S, box_in, kBN))
         return cudaErrorInvalidValue;
 
     GemmArgs g{};

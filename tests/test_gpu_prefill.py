@@ -35,6 +35,7 @@ SMALL = [
     (4, 1, 64, 2048, 64, 1, 8),
     (4, 1, 64, 300, 300, 512, 8),
     (32, 8, 64, 8192, 384, 2048, 8),
+    (8, 2, 64, 6000, 200, 2048, 8),
 ]
 
 
