@@ -10,7 +10,7 @@
 //   1. sample pass: only every S-th key column. A per-row radix select over
 //      those samples gives a threshold theta_row that about 1.75 B of the
 //      row's keys exceed;
-//   2. filter pass: all causal columns; the epilogue appends (key, position)
+//   2. filter pass: all causal columns; the epilogue appends (score, position)
 //      of every score >= theta_row to a per-row candidate list.
 // A final per-row selection takes the exact top B of the candidates (ties:
 // lower position) and writes them in ascending order through a position
@@ -144,7 +144,7 @@ struct GemmArgs {
     long long ld_samp;
     const uint32_t* thr;   // filter mode: [rows] order-key thresholds
     unsigned* cnt;         // [rows, 2 * nseg] per-writer counts
-    uint2* cand;           // [rows, cap] (key, position)
+    uint2* cand;           // [rows, ld_cand] (fp32 score bits, position)
     int cap_pair;          // entries per writer pair region
     long long ld_cand;     // entries per row = nseg * cap_pair
     unsigned* status;
@@ -350,7 +350,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // filter mode: this thread's writer slot and list region
             const int slot = half * a.nseg + un.seg;
             const bool down = (slot & 1) != 0;
-            uint2* region = a.cand + grow * a.ld_cand + (long long)(slot >> 1) * a.cap_pair;
+            // this writer's next list entry: upward from the region start, or
+            // downward from its end (entries hold the raw fp32 score bits)
+            uint2* wp = a.cand + grow * a.ld_cand + (long long)(slot >> 1) * a.cap_pair + (down ? a.cap_pair - 1 : 0);
+            const int dir = down ? -1 : 1;
             float thr_f = 0.f;
             if (MODE == kModeFilter) thr_f = vrow ? key_floor(__ldg(&a.thr[grow])) : __int_as_float(0x7f800000);
             unsigned n = 0;
@@ -413,14 +416,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                     st4[g] = make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
                                                          __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
                                 __syncwarp();
+                                // two passes per iteration: their shared-memory reads overlap
+                                const uint32_t* srow = reinterpret_cast<const uint32_t*>(stage + lane * kStageRow);
                                 while (m) {
-                                    const int j = __ffs(m) - 1;
+                                    const int j1 = __ffs(m) - 1;
                                     m &= m - 1u;
-                                    if (n < (unsigned)a.cap_pair) {
-                                        const unsigned at = down ? (unsigned)a.cap_pair - 1u - n : n;
-                                        region[at] = make_uint2(score_key(stage[lane * kStageRow + j]), (uint32_t)(cb + j));
-                                    }
+                                    const int j2 = m ? __ffs(m) - 1 : j1;
+                                    const bool two = m != 0u;
+                                    if (two) m &= m - 1u;
+                                    const uint32_t x1 = srow[j1], x2 = srow[j2];
+                                    if (n < (unsigned)a.cap_pair) *wp = make_uint2(x1, (uint32_t)(cb + j1));
+                                    wp += dir;
                                     ++n;
+                                    if (two) {
+                                        if (n < (unsigned)a.cap_pair) *wp = make_uint2(x2, (uint32_t)(cb + j2));
+                                        wp += dir;
+                                        ++n;
+                                    }
                                 }
                                 __syncwarp();
                             }
@@ -775,7 +787,7 @@ __global__ void __launch_bounds__(kSelThreads) prefill_select_kernel(const SelAr
             pp[it] = 0u;
             if (i < items) {
                 const uint2 e = entry(i);
-                kk[it] = e.x;
+                kk[it] = score_key(__uint_as_float(e.x));
                 pp[it] = e.y;
             }
         }
@@ -791,7 +803,7 @@ __global__ void __launch_bounds__(kSelThreads) prefill_select_kernel(const SelAr
             [&](auto f) {
                 for (int i = threadIdx.x; i < items; i += kSelThreads) {
                     const uint2 e = entry(i);
-                    f(e.x, e.y);
+                    f(score_key(__uint_as_float(e.x)), e.y);
                 }
             },
             need, n, sh, bitmap, out, a.B);
