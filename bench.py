@@ -247,6 +247,23 @@ def run_reference(args, rank, world):
         return 0
     from indexed_sparse_attention_kv_b200 import inputs as I
 
+    if args.workload in RESIDENT_METRICS:
+        w = I.workload(args.workload)
+        x = I.make_decode_inputs(w)
+        cpu_unit_sample(w, x, budget_s=0.0, max_units=max(1, args.warmup))
+        v, n, el = cpu_unit_sample(w, x, budget_s=0.0, max_units=max(1, args.steps))
+        line = {
+            "impl": "reference", "metric": RESIDENT_METRICS[w.name], "value": v, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "d": w.d, "T": w.T,
+                       "r": w.r, "B": w.B, "blk": w.blk, "keep": w.keep},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{n} (sequence, KV head) units per timed run, scaled to whole steps"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return 0
     if args.workload == "prefill_128k":
         w = I.workload("prefill_128k")
         x = I.make_prefill_inputs(w)
@@ -446,6 +463,185 @@ def run_ours(args, rank, world, local_rank):
                     "h2d_bytes_per_step": hq.numel() * 2 + hqt.numel() * 2,
                     "d2h_bytes_per_step": hout.numel() * 2 + hidx.numel() * 4},
             "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "clocks": clocks,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+RESIDENT_METRICS = {
+    "llama8b_32k": "sparse decode steps/s per layer at 32K, B=512 (LLaMA-3.1-8B layer shape)",
+    "hier_1m": "coarse-to-fine sparse decode steps/s per layer at 1M tokens (64-token blocks, keep 64, B=2048)",
+}
+
+
+def resident_bytes(w):
+    """Algorithmic bytes of one decode step: flat mode streams the projected-key
+    cache; coarse-to-fine mode reads the centroids and the kept blocks' projected
+    keys; both read the selected K/V rows and q, q~, out."""
+    small = w.batch * w.hq * (w.d * 2 + w.r * 2 + w.d * 2)
+    kv = w.batch * w.hkv * w.B * w.d * 2 * 2
+    if w.blk:
+        nblk = -(-w.T // w.blk)
+        score = w.batch * nblk * w.hkv * w.r * 2 + w.batch * w.keep * w.blk * w.hkv * w.r * 2
+    else:
+        score = w.batch * w.T * w.hkv * w.r * 2
+    return score + kv + small
+
+
+def cpu_unit_sample(w, x, budget_s=12.0, max_units=None):
+    """The oracle on (sequence, KV head) units of a decode step (flat or
+    coarse-to-fine) until about budget_s seconds; returns (steps/s, units, s)."""
+    import numpy as np
+    import torch
+
+    import oracle.lsa_oracle as O
+
+    units_per_step = w.batch * w.hkv
+    done, elapsed = 0, 0.0
+    while True:
+        b = (done // w.hkv) % w.batch
+        h = done % w.hkv
+        qt = x["qt"][b, h * w.G:(h + 1) * w.G].to(torch.float32).numpy()
+        kt = x["kt"][b, :, h:h + 1].to(torch.float32).numpy()
+        q = x["q"][b, h * w.G:(h + 1) * w.G].to(torch.float32).numpy()
+        ts = time.perf_counter()
+        q_bar = O.group_mean_query(qt, 1)
+        if w.blk:
+            idx = O.hierarchical_select(q_bar, kt, w.blk, w.keep, w.B)
+        else:
+            idx = O.select_top_b(O.candidate_scores(q_bar, kt)[0], w.B)[None]
+        sel = idx[0][idx[0] >= 0]
+        k_rows = x["k"][b, sel, h:h + 1].to(torch.float32).numpy()
+        v_rows = x["v"][b, sel, h:h + 1].to(torch.float32).numpy()
+        O.indexed_attention(q, k_rows, v_rows, np.arange(len(sel))[None], w.scale)
+        elapsed += time.perf_counter() - ts
+        done += 1
+        if elapsed >= budget_s or (max_units and done >= max_units):
+            break
+    return done / units_per_step / elapsed, done, elapsed
+
+
+def run_resident(args, rank, world, local_rank):
+    """Decode workloads whose per-step data fits in L2 (32K flat, 1M
+    coarse-to-fine): every timed step is followed by a 256 MiB L2 flush, and
+    the flush, timed alone the same way, is subtracted."""
+    import torch
+    import torch.distributed as dist
+
+    import indexed_sparse_attention_kv_b200 as lsa
+    from indexed_sparse_attention_kv_b200 import _lib
+    from indexed_sparse_attention_kv_b200 import inputs as I
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    lsa.lib()
+    w = I.workload(args.workload)
+    x = I.make_decode_inputs(w, seed=rank_seed(w, rank))
+    d = {k: x[k].to(dev) for k in ("q", "qt", "k", "v", "kt")}
+    dims = _lib.decode_dims(d["q"], d["qt"], d["k"])
+    cen = lsa.lsa_block_centroids(d["kt"], w.blk) if w.blk else None   # maintained offline, outside the step
+    ws = lsa.workspace(dims, w.B, w.blk, w.keep if w.blk else 0, device=dev)
+    idx = torch.empty((w.batch, w.hkv, w.B), dtype=torch.int32, device=dev)
+    out = torch.empty_like(d["q"])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lsa.lsa_decode_step(d["q"], d["qt"], d["k"], d["v"], d["kt"], w.B, centroids=cen, blk=w.blk,
+                            keep=w.keep, idx_out=idx, out=out, ws=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    status = lsa.lsa_read_device_status(ws)
+
+    def graph_of(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        g.replay()
+        torch.cuda.synchronize()
+        return g
+
+    def step_flush():
+        step()
+        flush.zero_()
+
+    g_sf = graph_of(step_flush)
+    g_f = graph_of(lambda: flush.zero_())
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+
+    def timed(g):
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return e0.elapsed_time(e1)
+
+    for _ in range(max(3, args.warmup)):
+        g_sf.replay()
+    with ClockSampler(dev) as clk:
+        ms_sf = timed(g_sf)
+    ms_f = timed(g_f)
+    clocks = clk.summary()
+    ms = max(1e-6, ms_sf - ms_f)
+    # end to end through the public API: H2D q, qt; step; D2H out, idx (flush after each, subtracted)
+    hq, hqt = x["q"].pin_memory(), x["qt"].pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hidx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        d["q"].copy_(hq, non_blocking=True)
+        d["qt"].copy_(hqt, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+        hidx.copy_(idx, non_blocking=True)
+        flush.zero_()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = max(1e-6, e0.elapsed_time(e1) - ms_f)
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        step_bytes = resident_bytes(w)
+        achieved = step_bytes / (ms / args.steps / 1e3) / 1e9
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            v, n, el = cpu_unit_sample(w, x, budget_s=args.cpu_budget)
+            cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                   "sample": f"{n} (sequence, KV head) units of {w.batch * w.hkv} per step ({el:.1f} s), scaled"}
+        line = {
+            "metric": RESIDENT_METRICS[w.name], "value": weak_value(world, args.steps, ms), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "d": w.d, "T": w.T,
+                       "r": w.r, "B": w.B, "blk": w.blk, "keep": w.keep,
+                       "l2": "256 MiB L2 flush after every step, timed alone and subtracted",
+                       "parallelism": f"replicas{world}" if world > 1 else "single"},
+            "roofline": {"bound": "hbm", "kernel": "lsa_decode_step (whole step)", "achieved": achieved,
+                         "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": step_bytes,
+                         "avg_launch_ms": ms / args.steps},
+            "cpu_baseline": cpu,
+            "e2e": {"value": weak_value(world, args.steps, ms_e2e), "unit": UNIT,
+                    "h2d_bytes_per_step": hq.numel() * 2 + hqt.numel() * 2,
+                    "d2h_bytes_per_step": hout.numel() * 2 + hidx.numel() * 4},
+            "gpu_launches": (5 if w.blk else 3) * args.steps,
             "clocks": clocks,
             "device_status": status,
         }
@@ -654,8 +850,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["decode_128k", "prefill_128k"], default="decode_128k",
-                    help="decode_128k (the headline) or prefill_128k (indexer + indexed attention)")
+    ap.add_argument("--workload", choices=["decode_128k", "prefill_128k", "llama8b_32k", "hier_1m"],
+                    default="decode_128k",
+                    help="decode_128k (the headline), prefill_128k (indexer + indexed attention), or the "
+                         "L2-resident decode steps llama8b_32k and hier_1m")
     ap.add_argument("--ncu-case", choices=["score", "topk", "attn", "step"], default=None,
                     help="run one component on a reduced 128K case (batch 2) for an ncu capture; no JSON")
     args = ap.parse_args(argv)
@@ -678,6 +876,8 @@ def main(argv=None):
     try:
         if args.workload == "prefill_128k":
             return run_prefill(args, rank, world, local_rank)
+        if args.workload in RESIDENT_METRICS:
+            return run_resident(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
