@@ -27,6 +27,7 @@
 // compaction over the keys themselves, with the same result.
 #include <cooperative_groups.h>
 
+#include "block_select.cuh"
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
 
@@ -555,6 +556,55 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster_kernel(const Top
     cluster.sync();   // keep this CTA's shared memory alive for remote readers
 }
 
+// Rows of at most NT * kSmallItems keys: one CTA per row holds the whole row
+// in registers and runs the exact block selection (radix passes on the order
+// keys, boundary ties to the lower position, ascending output through a
+// bitmap). Positions of coarse-to-fine candidates map through blkmap.
+constexpr int kSmallItems = 16;
+
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_small_kernel(const TopkArgs a) {
+    __shared__ BlockSelShared sh;
+    extern __shared__ uint32_t sbitmap[];
+    const int row = blockIdx.x;
+    const float* src = a.scores + (size_t)row * a.n;
+    pdl_launch_dependents();
+    pdl_wait();   // the scores come from the previous kernel
+    uint32_t kk[kSmallItems];
+#pragma unroll
+    for (int it = 0; it < kSmallItems; ++it) {
+        const int i = (int)threadIdx.x + it * NT;
+        kk[it] = i < a.n ? score_key(__ldcg(src + i)) : 0u;
+    }
+    if (a.ghist)   // the scorer's histogram is not needed here; leave it zero for the next step
+        for (int i = threadIdx.x; i < kBins; i += NT) a.ghist[(size_t)row * kBins + i] = 0u;
+    const int32_t* bm = a.blkmap ? a.blkmap + (size_t)row * a.keep : nullptr;
+    select_and_emit<NT>(
+        [&](auto f) {
+#pragma unroll
+            for (int it = 0; it < kSmallItems; ++it)
+                if (kk[it]) f(kk[it], (uint32_t)((int)threadIdx.x + it * NT));
+        },
+        a.B, a.n, sh, sbitmap, a.idx + (size_t)row * a.B,
+        a.B, [&](int i) -> int32_t { return bm ? bm[i / a.blk] * a.blk + i % a.blk : i; });
+}
+
+template <int NT>
+cudaError_t launch_small(const LaunchCtx& ctx, const TopkArgs& a, int rows) {
+    const int smem = (a.n + 31) / 32 * 4;
+    auto kern = topk_small_kernel<NT>;
+    cudaError_t e = ensure_dyn_smem((const void*)kern, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)rows);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = ctx.stream;
+    e = cudaLaunchKernelEx(&cfg, kern, a);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int n, int B, int32_t* idx,
@@ -568,6 +618,9 @@ cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int
     a.B = B;
     a.blk = blk;
     a.keep = keep;
+    if (n <= 256 * kSmallItems) return launch_small<256>(ctx, a, rows);
+    if (n <= 512 * kSmallItems) return launch_small<512>(ctx, a, rows);
+    if (n <= 1024 * kSmallItems) return launch_small<1024>(ctx, a, rows);
     // Cluster size: about 16K keys per CTA, at most 8 (portable); fewer CTAs
     // per row when there are many rows.
     int cs = 1;
