@@ -191,6 +191,8 @@ __global__ void __launch_bounds__(256) score_fine_kernel(const FineArgs a) {
 #pragma unroll
             for (int k = 0; k < 8; ++k) q[k] += __uint_as_float(((uint32_t)src[(size_t)g * R + k]) << 16);
     }
+    pdl_launch_dependents();
+    pdl_wait();   // the kept block ids come from the previous kernel
     const int32_t* bi = a.blk_idx + ((size_t)b * a.hkv + h) * a.keep;
     float* out = a.out + ((size_t)b * a.hkv + h) * a.ncand;
     const size_t row_stride = (size_t)a.hkv * R * 2;
@@ -470,11 +472,23 @@ cudaError_t launch_flat_r(const LaunchCtx& ctx, const ScoreArgs& a, int batch) {
 template <int R>
 cudaError_t launch_fine_r(const LaunchCtx& ctx, const FineArgs& a, int batch) {
     constexpr int TPW = 32 / (R / 8);
-    const int per_cta_target = 8 * TPW * 8;   // eight warp passes per warp
+    // one pass per warp: its two dependent loads (block id, then the row) are
+    // the whole latency chain
+    const int per_cta_target = 8 * TPW;
     int ctas = (a.ncand + per_cta_target - 1) / per_cta_target;
     if (ctas < 1) ctas = 1;
-    dim3 grid((unsigned)ctas, (unsigned)a.hkv, (unsigned)batch);
-    score_fine_kernel<R><<<grid, 256, 0, ctx.stream>>>(a);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)ctas, (unsigned)a.hkv, (unsigned)batch);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = ctx.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, score_fine_kernel<R>, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

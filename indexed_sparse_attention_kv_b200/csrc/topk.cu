@@ -600,6 +600,11 @@ cudaError_t launch_small(const LaunchCtx& ctx, const TopkArgs& a, int rows) {
     cfg.blockDim = dim3(NT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = ctx.stream;
+    cudaLaunchAttribute attr[1];   // prologue overlaps the previous kernel's tail
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
