@@ -623,8 +623,9 @@ cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int
     a.B = B;
     a.blk = blk;
     a.keep = keep;
-    if (n <= 256 * kSmallItems) return launch_small<256>(ctx, a, rows);
-    if (n <= 512 * kSmallItems) return launch_small<512>(ctx, a, rows);
+    // rows of up to 16K keys: one 1024-thread CTA per row (measured faster
+    // than 256 or 512 threads for 4K-key rows: the selection's passes and
+    // barriers, not the loads, set its time)
     if (n <= 1024 * kSmallItems) return launch_small<1024>(ctx, a, rows);
     // Cluster size: about 16K keys per CTA, at most 8 (portable); fewer CTAs
     // per row when there are many rows.
