@@ -38,7 +38,7 @@ constexpr int kEpiWarp0 = 4;
 constexpr int kEpiWarps = 8;
 constexpr int kAccCols = 2 * kBN;     // two accumulators (double-buffered)
 constexpr int kMaxStages = 6;
-constexpr int kSelThreads = 256;
+constexpr int kSelThreads = 512;
 constexpr int kMaxSamples = 8192;
 constexpr int kMaxSlots = 8;
 constexpr int kStageRow = 36;         // staging row pitch (floats): conflict-free 16-byte stores
@@ -580,7 +580,7 @@ __global__ void __launch_bounds__(kThrWarps * 32) prefill_threshold_kernel(const
 // loaded once into registers (kSelItems per thread); longer lists are read
 // from global memory on every pass, and rows re-done from scratch recompute
 // their scores.
-constexpr int kSelItems = 16;
+constexpr int kSelItems = 8;
 
 __global__ void __launch_bounds__(kSelThreads) prefill_select_kernel(const SelArgs a) {
     __shared__ SelShared sh;
