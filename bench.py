@@ -37,6 +37,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "sparse decode steps/s per layer at 128K, B=2048; achieved HBM GB/s vs peak"
+METRIC_FP8 = "sparse decode steps/s per layer at 128K, B=2048, FP8 (E4M3) projected-key cache; HBM GB/s vs peak"
 UNIT = "steps/s"
 WORKLOAD = "decode_128k"
 FALLBACK_HBM_GBS = 6650.0
@@ -294,7 +295,8 @@ def run_reference(args, rank, world):
     step_s = unit_s * w.batch * w.hkv
     value = 1.0 / step_s
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC_FP8 if args.workload == "decode_128k_fp8" else METRIC,
+        "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_dict(w),
@@ -317,9 +319,12 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     lsa.lib()
+    fp8 = args.workload == "decode_128k_fp8"
     w = I.workload(WORKLOAD)
     x = I.make_decode_inputs(w, seed=rank_seed(w, rank))
     d = {k: x[k].to(dev) for k in ("q", "qt", "k", "v", "kt")}
+    if fp8:   # the same integer values, stored as E4M3 (exact)
+        d["kt8"] = d["kt"].to(torch.float8_e4m3fn)
     dims = _lib.decode_dims(d["q"], d["qt"], d["k"])
     ws = lsa.workspace(dims, w.B, device=dev)
     idx = torch.empty((w.batch, w.hkv, w.B), dtype=torch.int32, device=dev)
@@ -327,7 +332,10 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        lsa.lsa_decode_step(d["q"], d["qt"], d["k"], d["v"], d["kt"], w.B, idx_out=idx, out=out, ws=ws)
+        if fp8:
+            lsa.lsa_decode_step_fp8(d["q"], d["qt"], d["k"], d["v"], d["kt8"], w.B, idx_out=idx, out=out, ws=ws)
+        else:
+            lsa.lsa_decode_step(d["q"], d["qt"], d["k"], d["v"], d["kt"], w.B, idx_out=idx, out=out, ws=ws)
 
     def barrier():
         if world > 1:
@@ -383,8 +391,10 @@ def run_ours(args, rank, world, local_rank):
         flush.zero_()
         lsa.lsa_indexed_attn(d["q"], d["k"], d["v"], idx, out=out, ws=ws)
 
+    score_call = (lambda: lsa.lsa_score_fp8(d["qt"], d["kt8"], scores)) if fp8 else \
+        (lambda: lsa.lsa_score(d["qt"], d["kt"], scores))
     graphs = {
-        "scoring": graph_of(lambda: lsa.lsa_score(d["qt"], d["kt"], scores), reps),
+        "scoring": graph_of(score_call, reps),
         "top_b": graph_of(lambda: lsa.lsa_topk(scores, w.B, idx), reps),
         "attention+flush": graph_of(attn_after_flush, reps),
         "flush": graph_of(lambda: flush.zero_(), reps),
@@ -434,11 +444,13 @@ def run_ours(args, rank, world, local_rank):
         value = weak_value(world, args.steps, ms)
         e2e = weak_value(world, args.steps, ms_e2e)
         kt_b, kv_b, small_b = algorithmic_bytes(w)
+        if fp8:
+            kt_b //= 2   # one byte per projected-key value
         peak, peak_kind = measured_peak()
         score_ms = comp[0]
         scorer_bytes = kt_b + w.batch * w.hq * w.r * 2
         achieved = scorer_bytes / (score_ms / 1e3) / 1e9
-        traffic = scorer_traffic(w)
+        traffic = None if fp8 else scorer_traffic(w)
         step_bytes = kt_b + kv_b + small_b
         step_gbs = step_bytes / (ms / args.steps / 1e3) / 1e9
         cpu = None
@@ -447,11 +459,14 @@ def run_ours(args, rank, world, local_rank):
             cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                    "sample": f"{n} (sequence, KV head) units of the 128K workload ({el:.1f} s), scaled to steps"}
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": METRIC_FP8 if fp8 else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_dict(w, {"parallelism": f"replicas{world}" if world > 1 else "single"}),
-            "roofline": {"bound": "hbm", "kernel": "score_q64_kernel (lsa_score)", "achieved": achieved, "peak": peak,
+            "config": config_dict(w, {"parallelism": f"replicas{world}" if world > 1 else "single",
+                                      **({"workload": "decode_128k_fp8", "kt_dtype": "fp8_e4m3"} if fp8 else {})}),
+            "roofline": {"bound": "hbm", "kernel": "score_q64_kernel (lsa_score_fp8)" if fp8 else
+                         "score_q64_kernel (lsa_score)", "achieved": achieved, "peak": peak,
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_kind": peak_kind, "algorithmic_bytes_per_launch": scorer_bytes,
                          "avg_launch_ms": score_ms},
@@ -850,10 +865,12 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["decode_128k", "prefill_128k", "llama8b_32k", "hier_1m"],
+    ap.add_argument("--workload", choices=["decode_128k", "decode_128k_fp8", "prefill_128k", "llama8b_32k",
+                                           "hier_1m"],
                     default="decode_128k",
-                    help="decode_128k (the headline), prefill_128k (indexer + indexed attention), or the "
-                         "L2-resident decode steps llama8b_32k and hier_1m")
+                    help="decode_128k (the headline), decode_128k_fp8 (the same step over an FP8 projected-key "
+                         "cache), prefill_128k (indexer + indexed attention), or the L2-resident decode steps "
+                         "llama8b_32k and hier_1m")
     ap.add_argument("--ncu-case", choices=["score", "topk", "attn", "step"], default=None,
                     help="run one component on a reduced 128K case (batch 2) for an ncu capture; no JSON")
     args = ap.parse_args(argv)

@@ -74,6 +74,7 @@ enum {
 };
 
 typedef uint16_t lsa_bf16;
+typedef uint8_t lsa_fp8_e4m3;   /* OCP FP8 E4M3 storage (1 byte per value) */
 
 /* Problem sizes. batch sequences, hq query heads, hkv KV heads, head dim d,
  * scoring-subspace rank r (the projected-key cache width), cache length T. */
@@ -182,6 +183,22 @@ LSA_API lsa_status lsa_decode_step(const lsa_dims* dims, const lsa_bf16* q, cons
                            const lsa_bf16* centroids, int blk, int nblk_keep, int B,
                            float scale, int32_t* idx_out, lsa_bf16* out,
                            void* ws, size_t ws_bytes, void* stream);
+
+/* FP8 projected-key cache (JSSA, Fig. 10: the projected-key cache may be held
+ * in FP8 while the KV cache and the attention stay in BF16). lsa_score and the
+ * flat-mode lsa_decode_step with kt [batch, T, hkv, r] stored as OCP FP8 E4M3,
+ * which halves the bytes the scorer streams. Every E4M3 value converts to fp32
+ * exactly, so scores and index sets equal those of a bf16 cache holding the
+ * same values (e.g. integers of magnitude at most 16, or multiples of 4 up to
+ * 32). r must be 64 and hkv one of 4, 8, 16, 32; other sizes return
+ * LSA_ERR_UNSUPPORTED. Workspace: lsa_workspace_size(dims, B, 0, 0). */
+LSA_API lsa_status lsa_score_fp8(const lsa_dims* dims, const lsa_bf16* qt, const lsa_fp8_e4m3* kt,
+                                 float* scores, void* stream);
+
+LSA_API lsa_status lsa_decode_step_fp8(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* qt,
+                                       const lsa_bf16* k, const lsa_bf16* v, const lsa_fp8_e4m3* kt, int B,
+                                       float scale, int32_t* idx_out, lsa_bf16* out, void* ws,
+                                       size_t ws_bytes, void* stream);
 
 /* Block centroids for coarse-to-fine scoring (LongCat Sparse Attention,
  * Abstract, strategy (3); Latent Sparse Attention, summary: queries score

@@ -12,6 +12,7 @@ from ._lib import (  # noqa: F401
     lsa_clear_device_status,
     lsa_debug_set_wait_limit,
     lsa_decode_step,
+    lsa_decode_step_fp8,
     lsa_dims,
     lsa_indexed_attn,
     lsa_indexed_attn_noalloc,
@@ -21,6 +22,7 @@ from ._lib import (  # noqa: F401
     prefill_workspace,
     lsa_read_device_status,
     lsa_score,
+    lsa_score_fp8,
     lsa_topk,
     lsa_workspace_size,
     workspace,

@@ -55,6 +55,8 @@ _SIGS = {
     "lsa_topk": (_I, [_DIMS, _P, _I, _P, _P, _SZ, _P]),
     "lsa_indexed_attn": (_I, [_DIMS, _P, _P, _P, _P, _I, ctypes.c_float, _P, _P, _SZ, _P]),
     "lsa_indexed_attn_noalloc": (_I, [_DIMS, _P, _P, _P, _P, _I, ctypes.c_float, _P, _P, _P]),
+    "lsa_score_fp8": (_I, [_DIMS, _P, _P, _P, _P]),
+    "lsa_decode_step_fp8": (_I, [_DIMS, _P, _P, _P, _P, _P, _I, ctypes.c_float, _P, _P, _P, _SZ, _P]),
     "lsa_decode_step": (_I, [_DIMS, _P, _P, _P, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _P, _SZ, _P]),
     "lsa_block_centroids": (_I, [_DIMS, _P, _I, _P, _P]),
     "lsa_prefill_workspace_size": (_SZ, [_DIMS, _I, _I]),
@@ -236,6 +238,52 @@ def lsa_decode_step(q, qt, k, v, kt, B: int, scale: float | None = None, centroi
     _check("lsa_decode_step", lib().lsa_decode_step(
         ctypes.byref(dims), _ptr(q), _ptr(qt), _ptr(k), _ptr(v), _ptr(kt), _ptr(centroids), int(blk), int(keep),
         int(B), ctypes.c_float(scale), _ptr(idx_out), _ptr(out), _ptr(ws), ws.numel(), _stream(q)))
+    return idx_out, out
+
+
+def _fp8(t, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (liblsa has no CPU path)")
+    if t.dtype != torch.float8_e4m3fn:
+        raise TypeError(f"{name} must be torch.float8_e4m3fn, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def lsa_score_fp8(qt: torch.Tensor, kt: torch.Tensor, scores: torch.Tensor | None = None) -> torch.Tensor:
+    """Group-mean scores [batch, hkv, T] of an FP8 E4M3 projected-key cache kt [batch, T, hkv, r]
+    (lsa.h: lsa_score_fp8)."""
+    _cuda(qt, "qt", torch.bfloat16)
+    _fp8(kt, "kt")
+    batch, T, hkv, r = kt.shape
+    dims = make_dims(batch, qt.shape[1], hkv, 128, r, T)
+    if scores is None:
+        scores = torch.empty((batch, hkv, T), dtype=torch.float32, device=kt.device)
+    _cuda(scores, "scores", torch.float32)
+    _check("lsa_score_fp8", lib().lsa_score_fp8(ctypes.byref(dims), _ptr(qt), _ptr(kt), _ptr(scores), _stream(kt)))
+    return scores
+
+
+def lsa_decode_step_fp8(q, qt, k, v, kt, B: int, scale: float | None = None, idx_out=None, out=None, ws=None,
+                        return_idx: bool = True):
+    """One flat decode step over an FP8 E4M3 projected-key cache (lsa.h: lsa_decode_step_fp8).
+    Returns (idx [batch, hkv, B] or None, out [batch, hq, d])."""
+    for t, n in ((q, "q"), (qt, "qt"), (k, "k"), (v, "v")):
+        _cuda(t, n, torch.bfloat16)
+    _fp8(kt, "kt")
+    dims = decode_dims(q, qt, k)
+    scale = 1.0 / math.sqrt(dims.d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if idx_out is None and return_idx:
+        idx_out = torch.empty((dims.batch, dims.hkv, B), dtype=torch.int32, device=q.device)
+    if idx_out is not None:
+        _cuda(idx_out, "idx_out", torch.int32)
+    if ws is None:
+        ws = workspace(dims, B, device=q.device)
+    _check("lsa_decode_step_fp8", lib().lsa_decode_step_fp8(
+        ctypes.byref(dims), _ptr(q), _ptr(qt), _ptr(k), _ptr(v), _ptr(kt), int(B), ctypes.c_float(scale),
+        _ptr(idx_out), _ptr(out), _ptr(ws), ws.numel(), _stream(q)))
     return idx_out, out
 
 

@@ -353,6 +353,53 @@ lsa_status lsa_decode_step(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf
     return from_cuda(e);
 }
 
+static bool fp8_shape_ok(const lsa_dims* d) {
+    return d->r == 64 && (d->hkv == 4 || d->hkv == 8 || d->hkv == 16 || d->hkv == 32);
+}
+
+lsa_status lsa_score_fp8(const lsa_dims* dims, const lsa_bf16* qt, const lsa_fp8_e4m3* kt, float* scores,
+                         void* stream) {
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if (!fp8_shape_ok(dims)) return LSA_ERR_UNSUPPORTED;
+    if (!qt || !kt || !scores) return LSA_ERR_ARG;
+    if (!aligned16(qt) || !aligned16(kt) || !aligned16(scores)) return LSA_ERR_ALIGN;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    return from_cuda(lsa::launch_score_fp8(ctx, qt, kt, scores, dims->batch, dims->hq, dims->hkv, dims->r, dims->T, 1,
+                                           nullptr));
+}
+
+lsa_status lsa_decode_step_fp8(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* qt, const lsa_bf16* k,
+                               const lsa_bf16* v, const lsa_fp8_e4m3* kt, int B, float scale, int32_t* idx_out,
+                               lsa_bf16* out, void* ws, size_t ws_bytes, void* stream) {
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if ((s = check_B(B)) != LSA_OK) return s;
+    if (!fp8_shape_ok(dims)) return LSA_ERR_UNSUPPORTED;
+    if (!q || !qt || !k || !v || !kt || !out) return LSA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(qt) || !aligned16(k) || !aligned16(v) || !aligned16(kt) || !aligned16(out))
+        return LSA_ERR_ALIGN;
+    if (idx_out && !aligned16(idx_out)) return LSA_ERR_ALIGN;
+    if (!std::isfinite(scale)) return LSA_ERR_ARG;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    const DecodeLayout L = decode_layout(dims, B, 0, 0, ctx.num_sms);
+    if ((s = check_ws(ws, ws_bytes, L.total)) != LSA_OK) return s;
+    unsigned* status = at<unsigned>(ws, L.status);
+    int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
+    bool hist = false;
+    uint32_t* gh = at<uint32_t>(ws, L.hist);
+    cudaError_t e = lsa::launch_score_fp8(ctx, qt, kt, at<float>(ws, L.scores), dims->batch, dims->hq, dims->hkv,
+                                          dims->r, dims->T, 0, status, gh, &hist);
+    if (e == cudaSuccess)
+        e = lsa::launch_topk(ctx, at<float>(ws, L.scores), dims->batch * dims->hkv, dims->T, B, idx, nullptr, 0, 0,
+                             hist ? gh : nullptr);
+    if (e == cudaSuccess)
+        e = lsa::launch_attn(ctx, L.plan, q, k, v, idx, B, scale, out, at<float>(ws, L.pm), at<float>(ws, L.pl),
+                             at<float>(ws, L.po), at<unsigned>(ws, L.counters), dims->batch, dims->hq, dims->hkv,
+                             dims->d, dims->T, (long long)dims->T * dims->hkv, status);
+    return from_cuda(e);
+}
+
 lsa_status lsa_block_centroids(const lsa_dims* dims, const lsa_bf16* kt, int blk, lsa_bf16* centroids, void* stream) {
     lsa_status s = check_dims(dims);
     if (s != LSA_OK) return s;

@@ -77,6 +77,12 @@ cudaError_t launch_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_
                          int hkv, int r, int n, int mode, unsigned* status, uint32_t* ghist = nullptr,
                          bool* hist_done = nullptr);
 
+// As launch_score with kt stored as OCP FP8 E4M3 (1 byte per value); r must be
+// 64 and hkv one of 4, 8, 16, 32 (else cudaErrorInvalidValue, nothing launched).
+cudaError_t launch_score_fp8(const LaunchCtx& ctx, const uint16_t* qt, const uint8_t* kt, float* out, int batch,
+                             int hq, int hkv, int r, int n, int mode, unsigned* status, uint32_t* ghist = nullptr,
+                             bool* hist_done = nullptr);
+
 cudaError_t launch_fine_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_t* kt, const int32_t* blk_idx,
                               int keep, int blk, float* out, int batch, int hq, int hkv, int r, int T);
 

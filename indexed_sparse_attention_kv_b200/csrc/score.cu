@@ -8,6 +8,9 @@
 // multi-stage shared-memory ring, and reduced with fp32 FMAs.
 #include <cuda_bf16.h>
 
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
 
@@ -23,7 +26,7 @@ constexpr long long kDrainNs = 4000000000ll;   // 4 s: copies in flight always l
 
 struct ScoreArgs {
     const uint16_t* qt;    // [batch, hq, r]
-    const uint8_t* kt;     // [batch, n, hkv, r] bf16
+    const uint8_t* kt;     // [batch, n, hkv, r] bf16 (or FP8 E4M3 for the FP8 scorer)
     float* out;            // [batch, hkv, n]
     int hq, hkv, n, G;
     int tok_per_chunk;     // tokens per stage, multiple of the tokens per warp pass
@@ -40,6 +43,28 @@ struct ScoreArgs {
 __device__ __forceinline__ float finalize_score(float acc, const ScoreArgs& a) {
     if (a.mode == 0) return acc;
     return a.g_pow2 ? acc * a.inv_g : __fdiv_rn(acc, (float)a.G);
+}
+
+// Two OCP FP8 E4M3 values (element 0 in the low byte) -> two floats (exact).
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// 16 E4M3 values . q[0..16), fp32 accumulation in channel order.
+__device__ __forceinline__ float dot16_e4m3(const uint4 w, const float* q) {
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f0 = e4m3x2_to_float2(ws[i]);
+        const float2 f1 = e4m3x2_to_float2(ws[i] >> 16);
+        acc = fmaf(q[4 * i + 0], f0.x, acc);
+        acc = fmaf(q[4 * i + 1], f0.y, acc);
+        acc = fmaf(q[4 * i + 2], f1.x, acc);
+        acc = fmaf(q[4 * i + 3], f1.y, acc);
+    }
+    return acc;
 }
 
 __device__ __forceinline__ float dot8(const uint4 w, const float* q) {
@@ -262,11 +287,14 @@ constexpr int kQThreads = (kQConsumers + 1) * 32;
 constexpr int kQChunk = 16384;
 constexpr int kHistBins = 2048;
 
-template <int STAGES, bool HIST>
+// FP8: the projected keys are OCP FP8 E4M3 (64 bytes per head row) instead of
+// bf16 (128 bytes); every lane then reads 32 channels as two 16-byte words.
+template <int STAGES, bool HIST, bool FP8>
 __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int hkv = a.hkv;
-    const int token_bytes = hkv * 128;
+    constexpr int kHeadBytes = FP8 ? 64 : 128;
+    const int token_bytes = hkv * kHeadBytes;
     const int tok = a.tok_per_chunk;
     uint8_t* stages = smem;
     float* qbar = reinterpret_cast<float*>(smem + STAGES * kQChunk);
@@ -336,11 +364,20 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
         const int half = lane & 1, tsub = (lane >> 1) & 3, hl = lane >> 3;
         const int head = q * 4 + hl;
         float qv[32];
+        if (FP8) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float* src = qbar + head * 64 + half * 32 + ((k + tsub) & 3) * 8;
+            for (int k = 0; k < 2; ++k) {
+                const float* src = qbar + head * 64 + half * 32 + ((k + tsub) & 1) * 16;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) qv[k * 8 + e] = src[e];
+                for (int e = 0; e < 16; ++e) qv[k * 16 + e] = src[e];
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float* src = qbar + head * 64 + half * 32 + ((k + tsub) & 3) * 8;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) qv[k * 8 + e] = src[e];
+            }
         }
         float* out_h = a.out + ((size_t)b * hkv + head) * a.n;
         const uint64_t keep_pol = policy_evict_last();   // the top-B selection re-reads the scores
@@ -353,20 +390,27 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
             }
             const int t0 = (c0 + i) * tok;
             const int ntok = min(tok, a.n - t0);
-            const uint8_t* st = stages + s * kQChunk + head * 128 + half * 64;
+            const uint8_t* st = stages + s * kQChunk + head * kHeadBytes + half * (kHeadBytes / 2);
             for (int tg = warp / quads; tg * 4 < ntok; tg += wpq) {
                 const int t = tg * 4 + tsub;
                 float acc0 = 0.f, acc1 = 0.f;
                 if (t < ntok) {
                     const uint8_t* row = st + (size_t)t * token_bytes;
-                    const uint4 w0 = *reinterpret_cast<const uint4*>(row + ((0 + tsub) & 3) * 16);
-                    const uint4 w1 = *reinterpret_cast<const uint4*>(row + ((1 + tsub) & 3) * 16);
-                    const uint4 w2 = *reinterpret_cast<const uint4*>(row + ((2 + tsub) & 3) * 16);
-                    const uint4 w3 = *reinterpret_cast<const uint4*>(row + ((3 + tsub) & 3) * 16);
-                    acc0 = dot8(w0, qv + 0);
-                    acc1 = dot8(w1, qv + 8);
-                    acc0 += dot8(w2, qv + 16);
-                    acc1 += dot8(w3, qv + 24);
+                    if (FP8) {
+                        const uint4 w0 = *reinterpret_cast<const uint4*>(row + ((0 + tsub) & 1) * 16);
+                        const uint4 w1 = *reinterpret_cast<const uint4*>(row + ((1 + tsub) & 1) * 16);
+                        acc0 = dot16_e4m3(w0, qv + 0);
+                        acc1 = dot16_e4m3(w1, qv + 16);
+                    } else {
+                        const uint4 w0 = *reinterpret_cast<const uint4*>(row + ((0 + tsub) & 3) * 16);
+                        const uint4 w1 = *reinterpret_cast<const uint4*>(row + ((1 + tsub) & 3) * 16);
+                        const uint4 w2 = *reinterpret_cast<const uint4*>(row + ((2 + tsub) & 3) * 16);
+                        const uint4 w3 = *reinterpret_cast<const uint4*>(row + ((3 + tsub) & 3) * 16);
+                        acc0 = dot8(w0, qv + 0);
+                        acc1 = dot8(w1, qv + 8);
+                        acc0 += dot8(w2, qv + 16);
+                        acc1 += dot8(w3, qv + 24);
+                    }
                 }
                 float acc = acc0 + acc1;
                 acc += __shfl_xor_sync(0xffffffffu, acc, 1);
@@ -397,11 +441,11 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
     }
 }
 
-template <int STAGES, bool HIST>
+template <int STAGES, bool HIST, bool FP8>
 cudaError_t launch_q64_t(const LaunchCtx& ctx, ScoreArgs a, int batch) {
     const size_t smem = (size_t)STAGES * kQChunk + (size_t)a.hkv * 64 * 4 +
                         (HIST ? (size_t)a.hkv * kHistBins / 2 * 4 : 0) + 2 * STAGES * 8 + 16;
-    auto kern = score_q64_kernel<STAGES, HIST>;
+    auto kern = score_q64_kernel<STAGES, HIST, FP8>;
     cudaError_t e = ensure_dyn_smem((const void*)kern, (int)smem);
     if (e != cudaSuccess) return e;
     int occ = 0;
@@ -420,8 +464,8 @@ cudaError_t launch_q64_t(const LaunchCtx& ctx, ScoreArgs a, int batch) {
 
 // Returns whether the histogram was produced (a.ghist non-null, hkv <= 8 and at
 // most 65535 tokens per CTA so that 16-bit shared counters cannot overflow).
-cudaError_t launch_q64(const LaunchCtx& ctx, ScoreArgs a, int batch, bool* hist_done) {
-    const int token_bytes = a.hkv * 128;
+cudaError_t launch_q64(const LaunchCtx& ctx, ScoreArgs a, int batch, bool* hist_done, bool fp8 = false) {
+    const int token_bytes = a.hkv * (fp8 ? 64 : 128);
     a.tok_per_chunk = kQChunk / token_bytes;
     a.chunks_per_batch = (a.n + a.tok_per_chunk - 1) / a.tok_per_chunk;
     bool hist = a.ghist != nullptr && a.hkv <= 8;
@@ -433,7 +477,8 @@ cudaError_t launch_q64(const LaunchCtx& ctx, ScoreArgs a, int batch, bool* hist_
         hist = max_chunks * a.tok_per_chunk <= 65535;
     }
     *hist_done = hist;
-    return hist ? launch_q64_t<4, true>(ctx, a, batch) : launch_q64_t<6, false>(ctx, a, batch);
+    if (fp8) return hist ? launch_q64_t<4, true, true>(ctx, a, batch) : launch_q64_t<6, false, true>(ctx, a, batch);
+    return hist ? launch_q64_t<4, true, false>(ctx, a, batch) : launch_q64_t<6, false, false>(ctx, a, batch);
 }
 
 template <int R, bool FIXED>
@@ -521,6 +566,29 @@ cudaError_t launch_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_
         case 128: return launch_flat_r<128>(ctx, a, batch);
         default: return cudaErrorInvalidValue;
     }
+}
+
+cudaError_t launch_score_fp8(const LaunchCtx& ctx, const uint16_t* qt, const uint8_t* kt, float* out, int batch,
+                             int hq, int hkv, int r, int n, int mode, unsigned* status, uint32_t* ghist,
+                             bool* hist_done) {
+    if (hist_done) *hist_done = false;
+    if (r != 64 || !(hkv == 4 || hkv == 8 || hkv == 16 || hkv == 32)) return cudaErrorInvalidValue;
+    ScoreArgs a{};
+    a.qt = qt;
+    a.kt = kt;
+    a.out = out;
+    a.hq = hq;
+    a.hkv = hkv;
+    a.n = n;
+    a.G = hq / hkv;
+    a.mode = mode;
+    a.g_pow2 = (a.G & (a.G - 1)) == 0;
+    a.inv_g = 1.0f / (float)a.G;
+    a.status = status;
+    a.wait_limit = ctx.wait_limit;
+    a.ghist = ghist;
+    bool dummy = false;
+    return launch_q64(ctx, a, batch, hist_done ? hist_done : &dummy, true);
 }
 
 cudaError_t launch_fine_score(const LaunchCtx& ctx, const uint16_t* qt, const uint16_t* kt, const int32_t* blk_idx,

@@ -127,3 +127,18 @@ def test_noalloc_rejects_before_any_device_use():
                                         ALIGNED, None, None) == -8
     assert lib.lsa_indexed_attn_noalloc(ctypes.byref(d), MISALIGNED, ALIGNED, ALIGNED, ALIGNED, 16, f(0.06),
                                         ALIGNED, None, None) == -2
+
+
+def test_fp8_validation():
+    lib = L.lib()
+    f = ctypes.c_float
+    for kw in (dict(r=32), dict(hq=8, hkv=2), dict(r=128, hkv=8, hq=32)):
+        d = _dims(**kw)
+        assert lib.lsa_score_fp8(ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, None) == -7
+        assert lib.lsa_decode_step_fp8(ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 16, f(0.1),
+                                       None, ALIGNED, ALIGNED, 1 << 40, None) == -7
+    d = _dims(hq=32, hkv=8)
+    assert lib.lsa_score_fp8(ctypes.byref(d), None, ALIGNED, ALIGNED, None) == -1
+    assert lib.lsa_score_fp8(ctypes.byref(d), ALIGNED, MISALIGNED, ALIGNED, None) == -2
+    assert lib.lsa_decode_step_fp8(ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 16, f(0.1),
+                                   None, ALIGNED, ALIGNED, 16, None) == -4
