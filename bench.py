@@ -843,8 +843,10 @@ def run_ncu_case(args):
     scores = lsa.lsa_score(d["qt"], d["kt"])
     idx = lsa.lsa_topk(scores, w.B)
     out = torch.empty_like(d["q"])
+    kt8 = d["kt"].to(torch.float8_e4m3fn) if args.ncu_case == "score8" else None
     fn = {
         "score": lambda: lsa.lsa_score(d["qt"], d["kt"], scores),
+        "score8": lambda: lsa.lsa_score_fp8(d["qt"], kt8, scores),
         "topk": lambda: lsa.lsa_topk(scores, w.B, idx),
         "attn": lambda: lsa.lsa_indexed_attn(d["q"], d["k"], d["v"], idx, out=out, ws=ws),
         "step": lambda: lsa.lsa_decode_step(d["q"], d["qt"], d["k"], d["v"], d["kt"], w.B, idx_out=idx, out=out,
@@ -871,7 +873,7 @@ def main(argv=None):
                     help="decode_128k (the headline), decode_128k_fp8 (the same step over an FP8 projected-key "
                          "cache), prefill_128k (indexer + indexed attention), or the L2-resident decode steps "
                          "llama8b_32k and hier_1m")
-    ap.add_argument("--ncu-case", choices=["score", "topk", "attn", "step"], default=None,
+    ap.add_argument("--ncu-case", choices=["score", "score8", "topk", "attn", "step"], default=None,
                     help="run one component on a reduced 128K case (batch 2) for an ncu capture; no JSON")
     args = ap.parse_args(argv)
     if args.ncu_case:

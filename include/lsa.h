@@ -210,7 +210,11 @@ LSA_API lsa_status lsa_decode_step_fp8(const lsa_dims* dims, const lsa_bf16* q, 
 LSA_API lsa_status lsa_block_centroids(const lsa_dims* dims, const lsa_bf16* kt, int blk,
                                lsa_bf16* centroids, void* stream);
 
-/* Bytes of workspace for lsa_prefill_index / lsa_prefill_attn. */
+/* Bytes of workspace for lsa_prefill_index / lsa_prefill_attn (one workspace
+ * serves both; calls that share it must not overlap on the GPU). The attention
+ * merge counters in it must be zero before the first lsa_prefill_attn (zero-fill
+ * the workspace once); every completed call leaves them at zero. Returns 0 for
+ * invalid sizes (batch != 1, nq < 1). */
 LSA_API size_t lsa_prefill_workspace_size(const lsa_dims* dims, int nq, int B);
 
 /* Prefill indexer (LongCat Sparse Attention, Abstract: the Lightning Indexer's
@@ -222,7 +226,11 @@ LSA_API size_t lsa_prefill_workspace_size(const lsa_dims* dims, int nq, int B);
  *   qt  [nq, hq, r]   bf16     kt [T, hkv, r] bf16
  *   idx [nq, hkv, B]  int32    out, ascending, -1 padded (rows with p+1 < B)
  * The group mean is rounded to bf16 for the tensor-core contraction (exact when
- * it is a multiple of 2^-k representable in bf16, e.g. integer inputs). */
+ * it is a multiple of 2^-k representable in bf16, e.g. integer inputs).
+ * Limits: T <= 2^18 (the per-row output bitmap lives in shared memory; larger
+ * caches return LSA_ERR_UNSUPPORTED). ws: lsa_prefill_workspace_size(dims, nq,
+ * B) bytes, 256-byte aligned, no initial value needed (its buffers are written
+ * before they are read); about 3.76 GiB for nq = 4096, T = 128K, B = 2048. */
 LSA_API lsa_status lsa_prefill_index(const lsa_dims* dims, const lsa_bf16* qt, int nq, int q_start,
                              const lsa_bf16* kt, int B, int32_t* idx,
                              void* ws, size_t ws_bytes, void* stream);
@@ -245,7 +253,7 @@ LSA_API lsa_status lsa_clear_device_status(void* ws, void* stream);
  * up and sets LSA_DEV_TIMEOUT (default 2e9; 0 = give up at the first failed
  * probe; negative restores the default). It affects only launches enqueued
  * after the call. Process-wide. */
-LSA_API void lsa_debug_set_wait_limit(long long polls);
+LSA_API void lsa_debug_set_wait_limit(long long ns);
 
 #ifdef __cplusplus
 }

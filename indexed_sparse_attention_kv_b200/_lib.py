@@ -371,5 +371,7 @@ def lsa_clear_device_status(ws: torch.Tensor) -> None:
     _check("lsa_clear_device_status", lib().lsa_clear_device_status(_ptr(ws), _stream(ws)))
 
 
-def lsa_debug_set_wait_limit(polls: int) -> None:
-    lib().lsa_debug_set_wait_limit(int(polls))
+def lsa_debug_set_wait_limit(ns: int) -> None:
+    """Device-time limit of every bounded wait in later launches (0: give up at the
+    first failed probe; negative: restore the default of 2 s)."""
+    lib().lsa_debug_set_wait_limit(int(ns))

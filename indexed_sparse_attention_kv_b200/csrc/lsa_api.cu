@@ -212,7 +212,7 @@ const char* lsa_status_string(lsa_status s) {
     }
 }
 
-void lsa_debug_set_wait_limit(long long polls) { g_wait_limit.store(polls < 0 ? kDefaultWaitLimit : polls); }
+void lsa_debug_set_wait_limit(long long ns) { g_wait_limit.store(ns < 0 ? kDefaultWaitLimit : ns); }
 
 size_t lsa_workspace_size(const lsa_dims* dims, int B, int blk, int nblk_keep) {
     if (check_dims(dims) != LSA_OK || check_B(B) != LSA_OK) return 0;

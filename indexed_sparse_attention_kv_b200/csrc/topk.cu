@@ -72,19 +72,6 @@ struct TopkShared {
     int total;
 };
 
-// Warp-level exclusive prefix sum; *total = the warp's sum.
-__device__ __forceinline__ int warp_excl_scan(int v, int* total) {
-    const int lane = threadIdx.x & 31;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    *total = __shfl_sync(0xffffffffu, x, 31);
-    return x - v;
-}
-
 // Given histogram `red` (nb bins) find the bin holding the krem-th largest
 // element counted from the top; sets sh.bstar and sh.above (count above it)
 // and returns the histogram total. All threads must call it.
