@@ -8,8 +8,8 @@
 // (tcgen05.mma, operands staged by TMA in 128-byte-swizzled shared memory,
 // fp32 accumulators in TMEM), twice:
 //   1. sample pass: only every S-th key column. A per-row radix select over
-//      those samples gives a threshold theta_row that about 1.75 B of the
-//      row's keys exceed;
+//      those samples gives a threshold theta_row that about 1.5 B of the
+//      row's keys exceed (a row left with fewer than B is re-selected, below);
 //   2. filter pass: all causal columns; the epilogue appends (score, position)
 //      of every score >= theta_row to a per-row candidate list.
 // A final per-row selection takes the exact top B of the candidates (ties:
@@ -730,7 +730,7 @@ PrefillPlan plan_prefill(int hq, int hkv, int r, int T, int nq, int B) {
     while (S * 2 <= B / 64) S *= 2;
     while (((long long)T + S - 1) / S > kMaxSamples) S *= 2;
     P.S = S;
-    P.kth = (int)((3LL * B + 2LL * S - 1) / (2LL * S)) + 16;    // ceil(1.5 B / S) + 16
+    P.kth = (int)((5LL * B + 4LL * S - 1) / (4LL * S)) + 16;    // ceil(1.25 B / S) + 16
     const long long expect = (long long)P.kth * S;               // keys expected above theta
     long long cap = 2 * expect;
     if (cap < B + B / 2 + 512) cap = B + B / 2 + 512;
