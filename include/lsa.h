@@ -230,7 +230,7 @@ LSA_API size_t lsa_prefill_workspace_size(const lsa_dims* dims, int nq, int B);
  * Limits: T <= 2^18 (the per-row output bitmap lives in shared memory; larger
  * caches return LSA_ERR_UNSUPPORTED). ws: lsa_prefill_workspace_size(dims, nq,
  * B) bytes, 256-byte aligned, no initial value needed (its buffers are written
- * before they are read); about 3.76 GiB for nq = 4096, T = 128K, B = 2048. */
+ * before they are read); about 3.26 GiB for nq = 4096, T = 128K, B = 2048. */
 LSA_API lsa_status lsa_prefill_index(const lsa_dims* dims, const lsa_bf16* qt, int nq, int q_start,
                              const lsa_bf16* kt, int B, int32_t* idx,
                              void* ws, size_t ws_bytes, void* stream);
