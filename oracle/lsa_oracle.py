@@ -29,7 +29,15 @@ Readings where the pages are silent (each is also listed in the design notes):
     selected positions, no RoPE/softcap/bias, and no forced sink/local tokens;
   * a block centroid is the sum of the projected keys of its (up to) ``blk``
     tokens, blocks starting at t = 0;
-  * prefill query at absolute position p sees keys 0 .. p inclusive.
+  * prefill query at absolute position p sees keys 0 .. p inclusive;
+  * scoring preparation (JSSA, Fig. 9 and Fig. 1, "a shared low-dimensional
+    subspace"): every KV head h has a basis P[h] of r vectors of length d; a
+    key of head h and the queries of h's group are both projected onto it,
+    y_j = <P[h, j], x> (one basis per layer is the case of equal P[h]). The
+    projected cache holds bf16 (round to nearest even, from the exact value)
+    or FP8 E4M3 (round to nearest even, saturated to +-448) values;
+  * a centroid maintained incrementally adds each new projected key to its
+    block in position order and rounds the sum to bf16 after every add.
 
 All parity statements in the tests hold against these functions. Parity pins
 (what fixes each function independently of itself) live in tests/test_oracle.py.
@@ -52,6 +60,12 @@ __all__ = [
     "prefill_scores",
     "prefill_index",
     "prefill_attention",
+    "round_to_bf16",
+    "round_to_e4m3",
+    "project_rows",
+    "project_bf16",
+    "project_e4m3",
+    "update_centroids",
 ]
 
 
@@ -250,3 +264,84 @@ def prefill_attention(q_rows, k, v, idx, scale: float) -> np.ndarray:
 
 def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
+
+
+# ---------------------------------------------------------------- scoring preparation
+def _round_to_grid(x, mant_bits: int, min_exp: int) -> np.ndarray:
+    """Round fp64 values to a binary format with `mant_bits` stored mantissa
+    bits and smallest normal exponent `min_exp`, ties to even; no overflow
+    handling (the callers clamp). Works on the exact fp64 value: one rounding."""
+    x = _f64(x)
+    out = np.zeros_like(x)
+    nz = (x != 0) & np.isfinite(x)
+    m, e = np.frexp(np.abs(x[nz]))         # |x| = m * 2**e, m in [0.5, 1)
+    e = np.maximum(e - 1, min_exp)         # exponent of the leading bit, or the subnormal floor
+    ulp = np.ldexp(1.0, e - mant_bits)
+    out[nz] = np.sign(x[nz]) * np.rint(np.abs(x[nz]) / ulp) * ulp   # np.rint: ties to even
+    out[~np.isfinite(x)] = x[~np.isfinite(x)]
+    return out
+
+
+def round_to_bf16(x) -> np.ndarray:
+    """Nearest bfloat16 value (8 exponent bits, 7 stored mantissa bits; ties
+    to even), as fp64. Values past the largest finite bf16 by half an ulp or
+    more become +-inf."""
+    y = _round_to_grid(x, 7, -126)
+    big = np.ldexp(2.0 - 2.0 ** -7, 127)
+    y[np.isfinite(y) & (np.abs(y) > big)] = np.sign(y[np.isfinite(y) & (np.abs(y) > big)]) * np.inf
+    return y
+
+
+def round_to_e4m3(x) -> np.ndarray:
+    """Nearest FP8 E4M3 value (4 exponent bits with bias 7, 3 stored mantissa
+    bits, largest finite 448, no infinities; ties to even), saturated to
+    +-448, as fp64."""
+    y = _round_to_grid(x, 3, -6)
+    return np.clip(y, -448.0, 448.0)
+
+
+def project_rows(x, P, G: int) -> np.ndarray:
+    """Exact projections y[..., i, j] = <P[i // G, j, :], x[..., i, :]> in fp64.
+
+    JSSA, Fig. 1 (a projected-key cache in a subspace shared with the scoring
+    query) and Fig. 9 (scoring preparation: the key projection). ``x`` is
+    [..., H, d] (keys: H = hkv, G = 1; queries: H = hq, G = hq / hkv), ``P`` is
+    [nbases, r, d] with H = nbases * G. Returns [..., H, r].
+    """
+    x = _f64(x)
+    P = _f64(P)
+    H, d = x.shape[-2:]
+    nb, r, dp = P.shape
+    assert dp == d and H == nb * G, "basis shape"
+    y = np.zeros(x.shape[:-1] + (r,), dtype=np.float64)
+    for i in range(H):
+        y[..., i, :] = x[..., i, :] @ P[i // G].T
+    return y
+
+
+def project_bf16(x, P, G: int) -> np.ndarray:
+    """The bf16 projected cache rows: round_to_bf16(project_rows(x, P, G))."""
+    return round_to_bf16(project_rows(x, P, G))
+
+
+def project_e4m3(x, P, G: int) -> np.ndarray:
+    """The FP8 E4M3 projected cache rows (JSSA, Fig. 10: the projected-key
+    cache held in FP8): round_to_e4m3(project_rows(x, P, G))."""
+    return round_to_e4m3(project_rows(x, P, G))
+
+
+def update_centroids(c, kt, t0: int, n: int, blk: int) -> np.ndarray:
+    """Incremental block centroids: for t = t0 .. t0+n-1 in order,
+    c[t // blk, h] <- round_to_bf16(c[t // blk, h] + kt[t, h]).
+
+    LongCat Sparse Attention, Abstract, strategy (3) Hierarchical Indexing (the
+    block-level keys of the coarse stage), kept current as tokens are appended
+    (JSSA, Fig. 9, scoring preparation). ``c`` is [nblk, hkv, r] (bf16 values),
+    ``kt`` is [T, hkv, r]. Returns the updated copy of ``c`` in fp64.
+    """
+    c = _f64(c).copy()
+    kt = _f64(kt)
+    for t in range(t0, t0 + n):
+        j = t // blk
+        c[j] = round_to_bf16(c[j] + kt[t])
+    return c

@@ -10,7 +10,12 @@
 * invariants (weights sum to 1, unselected rows never matter, keeping every
   block reduces coarse-to-fine to flat selection, block score == sum of token
   scores, a prefill row == decode selection over the row's causal prefix),
-* hand-derived worked examples under tests/golden/ (the pages print none).
+* hand-derived worked examples under tests/golden/ (the pages print none),
+* for scoring preparation: torch's fp32 -> bf16 / float8_e4m3fn casts on
+  values where one rounding is the whole story, hand-derived ties and
+  saturation, permuted unit bases (closed form), orthonormal bases
+  (Pythagoras), integer brute force, and incremental centroids that must
+  rebuild the (separately pinned) block sums.
 
 ``test_planted_mistakes_are_caught`` plants typical mistakes in copies of the
 oracle's functions and checks that at least one pin fails for every mistake.
@@ -283,11 +288,107 @@ def check_golden(o):
     assert np.array_equal(got, np.array(g["idx"]))
 
 
+# ------------------------------------------------------------------ scoring preparation
+
+def check_round_bf16(o):
+    """fp32-representable values: one rounding, so torch's fp32 -> bf16 cast
+    (round to nearest even) is the reference; plus hand-derived ties."""
+    rng = np.random.default_rng(21)
+    x32 = np.concatenate([rng.standard_normal(4000) * 10.0 ** rng.integers(-40, 38, 4000),
+                          rng.standard_normal(200) * 1e-39]).astype(np.float32)
+    x32 = x32[np.isfinite(x32)]
+    want = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(o.round_to_bf16(x32.astype(np.float64)), want)
+    # ulp 2 above 256: 257 and 259 are ties -> even mantissa; ulp 2^-7 at 1
+    hand = {257.0: 256.0, 259.0: 260.0, 1 + 2 ** -8: 1.0, 1 + 3 * 2 ** -8: 1 + 2 ** -6,
+            -(1 + 3 * 2 ** -8): -(1 + 2 ** -6), 1 + 2 ** -8 + 2 ** -30: 1 + 2 ** -7}
+    got = o.round_to_bf16(np.array(list(hand)))
+    assert np.array_equal(got, np.array(list(hand.values()))), got
+
+
+def check_round_e4m3(o):
+    """In-range fp32 values against torch's float8_e4m3fn cast; hand ties and
+    saturation at 448."""
+    rng = np.random.default_rng(22)
+    x32 = (rng.standard_normal(4000) * 2.0 ** rng.integers(-12, 8, 4000)).astype(np.float32)
+    x32 = x32[np.abs(x32) <= 448]
+    want = torch.from_numpy(x32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(o.round_to_e4m3(x32.astype(np.float64)), want)
+    # ulp 2 at 16: 17, 19 are ties; subnormal ulp 2^-9: 1.5 * 2^-9 is a tie -> 2^-8
+    hand = {17.0: 16.0, 19.0: 20.0, 1.5 * 2 ** -9: 2 ** -8, 1000.0: 448.0, -500.0: -448.0, 450.0: 448.0}
+    got = o.round_to_e4m3(np.array(list(hand)))
+    assert np.array_equal(got, np.array(list(hand.values()))), got
+
+
+def check_project_shifted_unit_basis(o):
+    """P[h, j] = unit vector e_{(j + 3h) mod d}: y[..., i, j] = x[..., i, (j + 3 (i // G)) mod d]
+    (closed form; fixes the group of head i and the orientation of the basis)."""
+    rng = np.random.default_rng(23)
+    for nb, G, d, r in [(2, 4, 16, 5), (3, 1, 6, 6), (4, 2, 8, 8)]:
+        H = nb * G
+        P = np.zeros((nb, r, d))
+        for h in range(nb):
+            for j in range(r):
+                P[h, j, (j + 3 * h) % d] = 1.0
+        x = rng.standard_normal((2, 3, H, d))
+        y = o.project_rows(x, P, G)
+        for i in range(H):
+            for j in range(r):
+                assert np.array_equal(y[..., i, j], x[..., i, (j + 3 * (i // G)) % d])
+
+
+def check_project_orthonormal(o):
+    """Orthonormal basis rows: ||P x||^2 + ||P' x||^2 = ||x||^2 for the complement P'."""
+    rng = np.random.default_rng(24)
+    d, r = 12, 5
+    Q, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    x = rng.standard_normal((7, 1, d))
+    y = o.project_rows(x, Q[:r][None], 1)
+    z = o.project_rows(x, Q[r:][None], 1)
+    assert np.allclose((y ** 2).sum(-1) + (z ** 2).sum(-1), (x ** 2).sum(-1), rtol=1e-12)
+
+
+def check_project_integer_exact(o):
+    """Small integers: the bf16 cache rows equal exact integer dot products
+    (|y| <= 32 is exact in bf16), brute force with Python ints."""
+    rng = np.random.default_rng(25)
+    nb, G, d, r = 2, 2, 16, 4
+    x = rng.integers(-2, 3, size=(3, nb * G, d))
+    P = rng.integers(-1, 2, size=(nb, r, d))
+    y = o.project_bf16(x, P, G)
+    for a in range(3):
+        for i in range(nb * G):
+            for j in range(r):
+                assert y[a, i, j] == sum(int(P[i // G, j, c]) * int(x[a, i, c]) for c in range(d))
+
+
+def check_update_centroids(o):
+    """Appending every token (in chunks) to zero centroids rebuilds the block
+    sums when they are exact; and a hand-derived rounding sequence: 256 + 1 +
+    1 + 3 in bf16 is 256, 256, 260 (each sum rounded: 257 and 259 are ties)."""
+    rng = np.random.default_rng(26)
+    T, hkv, r, blk = 37, 2, 3, 4
+    kt = rng.integers(-3, 4, size=(T, hkv, r)).astype(np.float64)
+    c = np.zeros(((T + blk - 1) // blk, hkv, r))
+    t = 0
+    for n in [5, 1, 0, 13, 18]:
+        c = o.update_centroids(c, kt, t, n, blk)
+        t += n
+    assert np.array_equal(c, o.block_centroids(kt, blk))
+    kt2 = np.array([[[0.0]], [[1.0]], [[1.0]], [[3.0]]])
+    c2 = o.update_centroids(np.array([[[256.0]]]), kt2, 1, 3, 4)
+    assert c2[0, 0, 0] == 260.0, c2
+    c3 = o.update_centroids(np.array([[[256.0]]]), kt2, 1, 2, 4)
+    assert c3[0, 0, 0] == 256.0, c3
+
+
 CHECKS = [
     check_select_bruteforce, check_select_special, check_scores_bruteforce, check_scores_onehot,
     check_attention_full_budget_sdpa, check_attention_subset_sdpa, check_attention_closed_forms,
     check_attention_unselected_irrelevant, check_centroids_closed_form, check_hier_reductions,
     check_prefill_vs_decode_prefix, check_golden,
+    check_round_bf16, check_round_e4m3, check_project_shifted_unit_basis, check_project_orthonormal,
+    check_project_integer_exact, check_update_centroids,
 ]
 
 
@@ -431,7 +532,65 @@ def _hier_block_upper_ties(q_bar, kt, blk, keep, B):
         q_bar, kt, blk, keep, B)
 
 
+def _bf16_truncate(x):                    # rounds toward zero
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(np.abs(x))
+    ulp = np.ldexp(1.0, np.maximum(e - 1, -126) - 7)
+    return np.sign(x) * np.floor(np.abs(x) / ulp) * ulp
+
+
+def _bf16_ties_away(x):                   # ties away from zero instead of to even
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(np.abs(x))
+    ulp = np.ldexp(1.0, np.maximum(e - 1, -126) - 7)
+    return np.sign(x) * np.floor(np.abs(x) / ulp + 0.5) * ulp
+
+
+def _e4m3_no_saturation(x):               # forgot the clamp to +-448
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(np.abs(x))
+    ulp = np.ldexp(1.0, np.maximum(e - 1, -6) - 3)
+    return np.sign(x) * np.rint(np.abs(x) / ulp) * ulp
+
+
+def _proj_i_mod_nb(x, P, G):              # head i uses basis i % nbases
+    x = np.asarray(x, dtype=np.float64)
+    P = np.asarray(P, dtype=np.float64)
+    H = x.shape[-2]
+    return np.stack([x[..., i, :] @ P[i % P.shape[0]].T for i in range(H)], axis=-2)
+
+
+def _proj_transposed(x, P, G):            # basis used as columns (P^T) instead of rows
+    x = np.asarray(x, dtype=np.float64)
+    P = np.asarray(P, dtype=np.float64)
+    H = x.shape[-2]
+    return np.stack([x[..., i, :] @ P[i // G] for i in range(H)], axis=-2)
+
+
+def _cent_round_once(c, kt, t0, n, blk):  # sums exactly, rounds once per block
+    c = np.asarray(c, dtype=np.float64).copy()
+    acc = c.copy()
+    for t in range(t0, t0 + n):
+        acc[t // blk] += np.asarray(kt[t], dtype=np.float64)
+    return O.round_to_bf16(acc)
+
+
+def _cent_wrong_block(c, kt, t0, n, blk):  # token t lands in block (t + 1) // blk
+    c = np.asarray(c, dtype=np.float64).copy()
+    for t in range(t0, t0 + n):
+        j = min((t + 1) // blk, c.shape[0] - 1)
+        c[j] = O.round_to_bf16(c[j] + np.asarray(kt[t], dtype=np.float64))
+    return c
+
+
 MUTANTS = {
+    "bf16_truncates": dict(round_to_bf16=_bf16_truncate),
+    "bf16_ties_away": dict(round_to_bf16=_bf16_ties_away),
+    "e4m3_not_saturated": dict(round_to_e4m3=_e4m3_no_saturation),
+    "projection_basis_i_mod_nbases": dict(project_rows=_proj_i_mod_nb),
+    "projection_basis_transposed": dict(project_rows=_proj_transposed),
+    "centroid_update_rounds_once": dict(update_centroids=_cent_round_once),
+    "centroid_update_wrong_block": dict(update_centroids=_cent_wrong_block),
     "group_i_mod_hkv": dict(group_mean_query=_gm_wrong_group),
     "group_sum_not_mean": dict(group_mean_query=_gm_sum),
     "ties_to_higher_position": dict(select_top_b=_sel_upper_ties),
