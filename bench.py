@@ -265,6 +265,23 @@ def run_reference(args, rank, world):
         }
         print(json.dumps(line), flush=True)
         return 0
+    if args.workload == "prepare_128k":
+        sh = PREPARE_SHAPE
+        hx = I.make_projection_inputs(PREPARE_SEED, 1, 4096, sh["H"], sh["d"], sh["r"], sh["H"], None, None)
+        cpu_prepare_sample(hx["x"], hx["P"], budget_s=0.0, max_tokens=256 * max(1, args.warmup))
+        v, n, el = cpu_prepare_sample(hx["x"], hx["P"], budget_s=0.0, max_tokens=256 * max(1, args.steps))
+        byt = prepare_bytes(sh)
+        line = {
+            "impl": "reference", "metric": PREPARE_METRIC, "value": v, "unit": PREPARE_UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": byt / (v * 1e9) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "prepare_128k", **sh, "nbases": sh["H"]},
+            "cpu_baseline": {"value": v, "unit": PREPARE_UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{n} token rows x 8 KV heads per timed run, same algorithmic bytes per row"},
+            "e2e": {"value": v, "unit": PREPARE_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return 0
     if args.workload == "prefill_128k":
         w = I.workload("prefill_128k")
         x = I.make_prefill_inputs(w)
@@ -825,6 +842,164 @@ def run_prefill(args, rank, world, local_rank):
     return 0
 
 
+PREPARE_METRIC = ("scoring preparation at 128K: projected-key cache build (batch 4 x 131072 tokens x 8 KV heads, "
+                  "d 128 -> r 64, bf16), HBM GB/s")
+PREPARE_UNIT = "GB/s"
+PREPARE_SHAPE = dict(batch=4, T=131072, H=8, d=128, r=64, hq=32)
+PREPARE_SEED = 1006
+
+
+def prepare_bytes(sh):
+    """Algorithmic bytes of one full projection: read x, write y, read the bases."""
+    rows = sh["batch"] * sh["T"] * sh["H"]
+    return rows * sh["d"] * 2 + rows * sh["r"] * 2 + sh["H"] * sh["r"] * sh["d"] * 2
+
+
+def cpu_prepare_sample(x, P, budget_s=12.0, max_tokens=None):
+    """Oracle projection of whole token rows (all heads) of sequence 0 until the
+    budget (or max_tokens) is spent; returns (GB/s of the algorithmic bytes, tokens, seconds)."""
+    import oracle.lsa_oracle as O
+
+    Pn = P.to(torch_float32()).numpy()
+    t0 = time.perf_counter()
+    n = 0
+    chunk = 256
+    while True:
+        xs = x[0, n:n + chunk].to(torch_float32()).numpy()
+        O.project_bf16(xs, Pn, 1)
+        n += xs.shape[0]
+        el = time.perf_counter() - t0
+        if (max_tokens is not None and n >= max_tokens) or (max_tokens is None and el >= budget_s):
+            break
+    sh = PREPARE_SHAPE
+    byt = n * sh["H"] * (sh["d"] * 2 + sh["r"] * 2)
+    return byt / el / 1e9, n, el
+
+
+def torch_float32():
+    import torch
+    return torch.float32
+
+
+def run_prepare(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import indexed_sparse_attention_kv_b200 as lsa
+    from indexed_sparse_attention_kv_b200 import inputs as I
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    lsa.lib()
+    sh = PREPARE_SHAPE
+    hx = I.make_projection_inputs(PREPARE_SEED + 7919 * rank, sh["batch"], sh["T"], sh["H"], sh["d"], sh["r"],
+                                  sh["H"], None, None)
+    x, P = hx["x"].to(dev), hx["P"].to(dev)
+    y = torch.empty((sh["batch"], sh["T"], sh["H"], sh["r"]), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lsa.lsa_project(x, P, y=y, dev_status=status)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = e0.elapsed_time(e1)
+    clocks = clk.summary()
+    # decode-time append: one new key row per (sequence, KV head), the step's
+    # 32 query rows, and the new key's block centroid
+    q = torch.randn((sh["batch"], 1, sh["hq"], sh["d"]), device=dev).to(torch.bfloat16)
+    qt = torch.empty((sh["batch"], 1, sh["hq"], sh["r"]), dtype=torch.bfloat16, device=dev)
+    cen = torch.zeros((sh["batch"], sh["T"] // 64, sh["H"], sh["r"]), dtype=torch.bfloat16, device=dev)
+
+    def append():
+        lsa.lsa_project(x, P, sh["T"] - 1, 1, y=y)
+        lsa.lsa_project(q, P, y=qt)
+        lsa.lsa_update_centroids(y, cen, 64, sh["T"] - 1, 1)
+
+    for _ in range(5):
+        append()
+    g = torch.cuda.CUDAGraph()
+    s2 = torch.cuda.Stream(dev)
+    s2.wait_stream(stream)
+    with torch.cuda.stream(s2):
+        append()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        append()
+    reps = 200
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    append_us = e0.elapsed_time(e1) / reps * 1e3
+    del g
+    # end to end: the cache rows from pinned host memory, the projections back
+    hxp = hx["x"].pin_memory()
+    hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    e2e_steps = max(1, min(args.steps, 10))
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x.copy_(hxp, non_blocking=True)
+        step()
+        hy.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = e0.elapsed_time(e1)
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
+    st = int(status.item())
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        byt = prepare_bytes(sh)
+        per_ms = ms / args.steps
+        achieved = byt / (per_ms / 1e3) / 1e9
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            v, n, el = cpu_prepare_sample(hx["x"], hx["P"], budget_s=args.cpu_budget)
+            cpu = {"value": v, "unit": PREPARE_UNIT, "cores": blas_threads(), "kind": "oracle",
+                   "sample": f"{n} token rows x 8 KV heads of sequence 0 ({el:.1f} s), same algorithmic bytes per row"}
+        line = {
+            "metric": PREPARE_METRIC, "value": achieved * world, "unit": PREPARE_UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": per_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "prepare_128k", **sh, "nbases": sh["H"],
+                       "l2": "inputs exceed L2 (1 GiB of keys per step)"},
+            "roofline": {"bound": "hbm", "kernel": "project_kernel (lsa_project)", "achieved": achieved,
+                         "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": byt, "avg_launch_ms": per_ms},
+            "append_us": append_us,
+            "cpu_baseline": cpu,
+            "e2e": {"value": prepare_bytes(sh) * e2e_steps / (ms_e2e / 1e3) / 1e9 * world, "unit": PREPARE_UNIT,
+                    "h2d_bytes_per_step": hxp.numel() * 2, "d2h_bytes_per_step": hy.numel() * 2},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "device_status": st,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ncu_case(args):
     """A small, self-contained launch sequence for ncu captures: batch 2 of the
     128K workload (kt 256 MiB > L2, 1.3 GiB on the device), `--steps` launches
@@ -835,6 +1010,16 @@ def run_ncu_case(args):
     from indexed_sparse_attention_kv_b200 import _lib
     from indexed_sparse_attention_kv_b200 import inputs as I
 
+    if args.ncu_case == "project":   # one sequence of the 128K projection (256 MiB of keys in)
+        sh = PREPARE_SHAPE
+        hx = I.make_projection_inputs(PREPARE_SEED, 1, sh["T"], sh["H"], sh["d"], sh["r"], sh["H"], None, None)
+        xd, Pd = hx["x"].cuda(), hx["P"].cuda()
+        y = torch.empty((1, sh["T"], sh["H"], sh["r"]), dtype=torch.bfloat16, device="cuda")
+        for _ in range(args.warmup + args.steps):
+            lsa.lsa_project(xd, Pd, y=y)
+        torch.cuda.synchronize()
+        print(f"ncu case project: {args.warmup}+{args.steps} launches")
+        return 0
     w = I.workload(WORKLOAD).with_(batch=2, name="decode_128k_b2")
     x = I.make_decode_inputs(w)
     d = {k: x[k].cuda() for k in ("q", "qt", "k", "v", "kt")}
@@ -868,12 +1053,13 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=["decode_128k", "decode_128k_fp8", "prefill_128k", "llama8b_32k",
-                                           "hier_1m"],
+                                           "hier_1m", "prepare_128k"],
                     default="decode_128k",
                     help="decode_128k (the headline), decode_128k_fp8 (the same step over an FP8 projected-key "
-                         "cache), prefill_128k (indexer + indexed attention), or the L2-resident decode steps "
-                         "llama8b_32k and hier_1m")
-    ap.add_argument("--ncu-case", choices=["score", "score8", "topk", "attn", "step"], default=None,
+                         "cache), prefill_128k (indexer + indexed attention), the L2-resident decode steps "
+                         "llama8b_32k and hier_1m, or prepare_128k (scoring preparation: projecting the 128K "
+                         "key cache, and the decode-time append)")
+    ap.add_argument("--ncu-case", choices=["score", "score8", "topk", "attn", "step", "project"], default=None,
                     help="run one component on a reduced 128K case (batch 2) for an ncu capture; no JSON")
     args = ap.parse_args(argv)
     if args.ncu_case:
@@ -895,6 +1081,8 @@ def main(argv=None):
     try:
         if args.workload == "prefill_128k":
             return run_prefill(args, rank, world, local_rank)
+        if args.workload == "prepare_128k":
+            return run_prepare(args, rank, world, local_rank)
         if args.workload in RESIDENT_METRICS:
             return run_resident(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)

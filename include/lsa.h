@@ -210,6 +210,50 @@ LSA_API lsa_status lsa_decode_step_fp8(const lsa_dims* dims, const lsa_bf16* q, 
 LSA_API lsa_status lsa_block_centroids(const lsa_dims* dims, const lsa_bf16* kt, int blk,
                                lsa_bf16* centroids, void* stream);
 
+/* ---- Scoring preparation (JSSA, Fig. 9: the key projection that fills the
+ * projected-key cache; Fig. 1: keys and the group's queries are scored in a
+ * shared low-dimensional subspace). Every basis P[j] holds r vectors of length
+ * d; row i of x uses basis i / G with G = H / nbases:
+ *   y[b, t, i, c] = sum_e P[i / G, c, e] * x[b, t, i, e]
+ * accumulated in fp32 on the tensor cores and rounded to nearest even once.
+ * Keys: x = k [batch, T, hkv, d], H = nbases = hkv, y = kt.
+ * Queries: x = q viewed as [batch, 1, hq, d] (T = 1, t0 = 0, n = 1),
+ *          nbases = hkv, y = qt viewed as [batch, 1, hq, r].
+ * (One basis per layer: nbases = 1.) */
+typedef struct lsa_proj_dims {
+    int batch, T, H, d, r, nbases;
+} lsa_proj_dims;
+
+/* Project rows t0 .. t0 + n - 1 of every sequence (0 <= t0, n >= 0,
+ * t0 + n <= T; n = 0 does nothing); other rows of y are left untouched.
+ *   x [batch, T, H, d] bf16   P [nbases, r, d] bf16   y [batch, T, H, r] bf16
+ * Sizes: H % nbases == 0; d a multiple of 16 with d in {16, 32} or
+ * 64 <= d <= 256; r a multiple of 16 in [16, 128]; batch * T < 2^31; other
+ * sizes return LSA_ERR_UNSUPPORTED (d = 256 with r above 80 does not fit the
+ * staging buffers). x, P, y 16-byte aligned.
+ * dev_status: NULL, or a caller-owned device int32 into which LSA_DEV_TIMEOUT
+ * is OR-ed if a bounded wait ran out. The call allocates nothing. */
+LSA_API lsa_status lsa_project(const lsa_proj_dims* dims, const lsa_bf16* x, const lsa_bf16* P, int t0,
+                               int n, lsa_bf16* y, int32_t* dev_status, void* stream);
+
+/* lsa_project with an FP8 E4M3 output (JSSA, Fig. 10: the projected-key cache
+ * held in FP8): each fp32 projection rounds to nearest even E4M3, saturated to
+ * +-448. y [batch, T, H, r] lsa_fp8_e4m3. */
+LSA_API lsa_status lsa_project_fp8(const lsa_proj_dims* dims, const lsa_bf16* x, const lsa_bf16* P, int t0,
+                                   int n, lsa_fp8_e4m3* y, int32_t* dev_status, void* stream);
+
+/* Incremental block centroids (LongCat Sparse Attention, Abstract, strategy
+ * (3)): for every sequence and KV head, add the projected keys of positions
+ * t0 .. t0 + n - 1 to the centroid of their block, in position order,
+ * rounding the sum to bf16 after every add:
+ *   centroids[b, t / blk, h, :] <- bf16(centroids[b, t / blk, h, :] + kt[b, t, h, :])
+ *   kt [batch, T, hkv, r] bf16 (dims.T = capacity), centroids [batch, ceil(T/blk), hkv, r]
+ * Starting from zeros and adding a block's tokens gives lsa_block_centroids'
+ * value whenever the partial sums are exact in bf16 (e.g. small integers).
+ * 0 <= t0, n >= 0, t0 + n <= T, blk in [1, 4096]. */
+LSA_API lsa_status lsa_update_centroids(const lsa_dims* dims, const lsa_bf16* kt, int blk, int t0, int n,
+                                        lsa_bf16* centroids, void* stream);
+
 /* Bytes of workspace for lsa_prefill_index / lsa_prefill_attn (one workspace
  * serves both; calls that share it must not overlap on the GPU). The attention
  * merge counters in it must be zero before the first lsa_prefill_attn (zero-fill

@@ -19,6 +19,10 @@ from ._lib import (  # noqa: F401
     lsa_prefill_attn,
     lsa_prefill_index,
     lsa_prefill_workspace_size,
+    lsa_proj_dims,
+    lsa_project,
+    lsa_project_fp8,
+    lsa_update_centroids,
     prefill_workspace,
     lsa_read_device_status,
     lsa_score,

@@ -43,6 +43,14 @@ class lsa_dims(ctypes.Structure):
         return "lsa_dims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
 
 
+class lsa_proj_dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+                ("d", ctypes.c_int), ("r", ctypes.c_int), ("nbases", ctypes.c_int)]
+
+    def __repr__(self):
+        return "lsa_proj_dims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _SZ = ctypes.c_size_t
@@ -59,6 +67,9 @@ _SIGS = {
     "lsa_decode_step_fp8": (_I, [_DIMS, _P, _P, _P, _P, _P, _I, ctypes.c_float, _P, _P, _P, _SZ, _P]),
     "lsa_decode_step": (_I, [_DIMS, _P, _P, _P, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _P, _SZ, _P]),
     "lsa_block_centroids": (_I, [_DIMS, _P, _I, _P, _P]),
+    "lsa_project": (_I, [ctypes.POINTER(lsa_proj_dims), _P, _P, _I, _I, _P, _P, _P]),
+    "lsa_project_fp8": (_I, [ctypes.POINTER(lsa_proj_dims), _P, _P, _I, _I, _P, _P, _P]),
+    "lsa_update_centroids": (_I, [_DIMS, _P, _I, _I, _I, _P, _P]),
     "lsa_prefill_workspace_size": (_SZ, [_DIMS, _I, _I]),
     "lsa_prefill_index": (_I, [_DIMS, _P, _I, _I, _P, _I, _P, _P, _SZ, _P]),
     "lsa_prefill_attn": (_I, [_DIMS, _P, _I, _P, _P, _P, _I, ctypes.c_float, _P, _P, _SZ, _P]),
@@ -297,6 +308,49 @@ def lsa_block_centroids(kt: torch.Tensor, blk: int, centroids=None) -> torch.Ten
     _cuda(centroids, "centroids", torch.bfloat16)
     _check("lsa_block_centroids", lib().lsa_block_centroids(ctypes.byref(dims), _ptr(kt), int(blk),
                                                             _ptr(centroids), _stream(kt)))
+    return centroids
+
+
+def _project(fn, x, P, t0, n, y, ydtype, dev_status):
+    _cuda(x, "x", torch.bfloat16)
+    _cuda(P, "P", torch.bfloat16)
+    if x.dim() != 4 or P.dim() != 3:
+        raise LsaError(fn, -1, "x must be [batch, T, H, d] and P [nbases, r, d]")
+    batch, T, H, d = x.shape
+    nbases, r, _ = P.shape
+    if y is None:
+        y = torch.zeros((batch, T, H, r), dtype=ydtype, device=x.device)
+    _cuda(y, "y", ydtype)
+    if dev_status is not None:
+        _cuda(dev_status, "dev_status", torch.int32)
+    dims = lsa_proj_dims(batch, T, H, d, r, nbases)
+    t0 = 0 if t0 is None else int(t0)
+    n = T - t0 if n is None else int(n)
+    _check(fn, getattr(lib(), fn)(ctypes.byref(dims), _ptr(x), _ptr(P), t0, n, _ptr(y), _ptr(dev_status),
+                                  _stream(x)))
+    return y
+
+
+def lsa_project(x, P, t0: int | None = None, n: int | None = None, y=None, dev_status=None) -> torch.Tensor:
+    """Project rows t0 .. t0+n-1 of x [batch, T, H, d] onto the bases P [nbases, r, d]
+    (row i uses basis i // (H // nbases)) into y [batch, T, H, r] bf16 (lsa.h: lsa_project)."""
+    return _project("lsa_project", x, P, t0, n, y, torch.bfloat16, dev_status)
+
+
+def lsa_project_fp8(x, P, t0: int | None = None, n: int | None = None, y=None, dev_status=None) -> torch.Tensor:
+    """lsa_project into an FP8 E4M3 y [batch, T, H, r] (lsa.h: lsa_project_fp8)."""
+    return _project("lsa_project_fp8", x, P, t0, n, y, torch.float8_e4m3fn, dev_status)
+
+
+def lsa_update_centroids(kt: torch.Tensor, centroids: torch.Tensor, blk: int, t0: int, n: int) -> torch.Tensor:
+    """Add kt rows t0 .. t0+n-1 [batch, T, hkv, r] to their block centroids
+    [batch, ceil(T/blk), hkv, r] in place, bf16 after every add (lsa.h: lsa_update_centroids)."""
+    _cuda(kt, "kt", torch.bfloat16)
+    _cuda(centroids, "centroids", torch.bfloat16)
+    batch, T, hkv, r = kt.shape
+    dims = make_dims(batch, hkv, hkv, 128, r, T)
+    _check("lsa_update_centroids", lib().lsa_update_centroids(ctypes.byref(dims), _ptr(kt), int(blk), int(t0),
+                                                              int(n), _ptr(centroids), _stream(kt)))
     return centroids
 
 

@@ -410,6 +410,49 @@ lsa_status lsa_block_centroids(const lsa_dims* dims, const lsa_bf16* kt, int blk
     return from_cuda(lsa::launch_centroids(ctx, kt, blk, centroids, dims->batch, dims->hkv, dims->r, dims->T));
 }
 
+static lsa_status project_common(const lsa_proj_dims* pd, const lsa_bf16* x, const lsa_bf16* P, int t0, int n,
+                                 void* y, bool fp8, int32_t* dev_status, void* stream) {
+    if (!pd || !x || !P || !y) return LSA_ERR_ARG;
+    if (pd->batch < 1 || pd->T < 1 || pd->H < 1 || pd->d < 1 || pd->r < 1 || pd->nbases < 1) return LSA_ERR_ARG;
+    if (pd->H % pd->nbases != 0) return LSA_ERR_ARG;
+    if (t0 < 0 || n < 0 || (long long)t0 + n > pd->T) return LSA_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(P) || !aligned16(y)) return LSA_ERR_ALIGN;
+    if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return LSA_ERR_ALIGN;
+    const int d = pd->d, r = pd->r;
+    const bool d_ok = d % 16 == 0 && (d == 16 || d == 32 || (d >= 64 && d <= 256));
+    const bool r_ok = r % 16 == 0 && r >= 16 && r <= 128;
+    if (!d_ok || !r_ok || (long long)pd->batch * pd->T >= (1ll << 31) || lsa::project_stages(d, r, 2) < 2)
+        return LSA_ERR_UNSUPPORTED;
+    if (n == 0) return LSA_OK;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    return from_cuda(lsa::launch_project(ctx, x, P, y, fp8, pd->batch, pd->T, pd->H, d, r, pd->nbases, t0, n,
+                                         reinterpret_cast<unsigned*>(dev_status)));
+}
+
+lsa_status lsa_project(const lsa_proj_dims* dims, const lsa_bf16* x, const lsa_bf16* P, int t0, int n, lsa_bf16* y,
+                       int32_t* dev_status, void* stream) {
+    return project_common(dims, x, P, t0, n, y, false, dev_status, stream);
+}
+
+lsa_status lsa_project_fp8(const lsa_proj_dims* dims, const lsa_bf16* x, const lsa_bf16* P, int t0, int n,
+                           lsa_fp8_e4m3* y, int32_t* dev_status, void* stream) {
+    return project_common(dims, x, P, t0, n, y, true, dev_status, stream);
+}
+
+lsa_status lsa_update_centroids(const lsa_dims* dims, const lsa_bf16* kt, int blk, int t0, int n,
+                                lsa_bf16* centroids, void* stream) {
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if (!kt || !centroids) return LSA_ERR_ARG;
+    if (blk < 1 || blk > 4096) return LSA_ERR_ARG;
+    if (t0 < 0 || n < 0 || (long long)t0 + n > dims->T) return LSA_ERR_SHAPE;
+    if (!aligned16(kt) || !aligned16(centroids)) return LSA_ERR_ALIGN;
+    if (n == 0) return LSA_OK;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    return from_cuda(lsa::launch_centroid_update(ctx, kt, centroids, dims->batch, dims->T, dims->hkv, dims->r, blk,
+                                                 t0, n));
+}
+
 size_t lsa_prefill_workspace_size(const lsa_dims* dims, int nq, int B) {
     if (check_dims(dims) != LSA_OK || check_B(B) != LSA_OK || nq < 1 || dims->batch != 1) return 0;
     return prefill_layout(dims, nq, B, device_sms()).total;

@@ -94,6 +94,19 @@ cudaError_t launch_centroids(const LaunchCtx& ctx, const uint16_t* kt, int blk, 
 cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int n, int B, int32_t* idx,
                         const int32_t* blkmap, int blk, int keep, uint32_t* ghist = nullptr);
 
+// Scoring preparation (project.cu). y[b, t, i, :] = P[i / (H / nbases)] x[b, t, i, :]
+// for t in [t0, t0 + n) of every sequence: x [batch, T, H, d] bf16, P
+// [nbases, r, d] bf16, y [batch, T, H, r] bf16 or FP8 E4M3 (fp8). Needs
+// d % 16 == 0 with d in {16, 32} or 64 <= d <= 256, r % 16 == 0 with
+// 16 <= r <= 128, and project_stages(d, r, 2) >= 2.
+int project_stages(int d, int r, long long ntiles);
+cudaError_t launch_project(const LaunchCtx& ctx, const uint16_t* x, const uint16_t* P, void* y, bool fp8, int batch,
+                           int T, int H, int d, int r, int nbases, int t0, int n, unsigned* status);
+// cen [batch, ceil(T / blk), hkv, r] bf16 += kt rows t0 .. t0+n-1 of every
+// sequence, in position order, rounding to bf16 after every add.
+cudaError_t launch_centroid_update(const LaunchCtx& ctx, const uint16_t* kt, uint16_t* cen, int batch, int T, int hkv,
+                                   int r, int blk, int t0, int n);
+
 AttnPlan plan_attn(int nb, int hkv, int G, int B, int d, int num_sms);
 
 // pm/pl: [units, smax, G] fp32, po: [units, smax, G, d] fp32, counters:

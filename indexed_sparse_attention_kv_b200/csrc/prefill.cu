@@ -27,6 +27,7 @@
 #include "block_select.cuh"
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
+#include "tcgen05.cuh"
 
 namespace lsa {
 namespace {
@@ -46,83 +47,9 @@ constexpr int kStageFloats = 32 * kStageRow;          // writer slots per row (2
 constexpr int kModeSample = 0;        // epilogue writes scores of sampled columns
 constexpr int kModeFilter = 1;        // epilogue appends scores above the row threshold
 
-// tcgen05.mma instruction descriptor, kind::f16: D fp32, A and B bf16, both
-// K-major, N = 256, M = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
-                            ((uint32_t)(kBM >> 4) << 24);
-
-// ---------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-            "r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)),
-                 "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Arrive once on `bar` when every tcgen05 operation this thread issued so far
-// has completed.
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_addr(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
-        : "memory");
-}
-
-// 32 consecutive fp32 columns of this warp's 32 TMEM lanes (lane i of the
-// warp gets TMEM lane base + i). The registers are valid after tmem_wait.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr));
-}
-// Wait for this thread's TMEM loads; the registers are tied to the wait so
-// that no use of them is scheduled before it.
-__device__ __forceinline__ void tmem_wait(uint32_t (&v)[32]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
-                   "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),
-                   "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
-                   "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]),
-                   "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
-                 :
-                 : "memory");
-}
-
-// Shared-memory matrix descriptor of a K-major operand tile in the swizzled
-// layout TMA writes: rows of `rb` bytes (32, 64 or 128 = the swizzle span),
-// 8-row atoms `8 * rb` bytes apart.
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t rb) {
-    const uint32_t layout = rb == 128 ? 2u : (rb == 64 ? 4u : 6u);
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) |
-           ((uint64_t)(((8u * rb) >> 4) & 0x3FFFu) << 32) | ((uint64_t)1u << 46) | ((uint64_t)layout << 61);
-}
+// tcgen05.mma instruction descriptor: D fp32, A and B bf16, both K-major,
+// M = 128, N = 256.
+constexpr uint32_t kIdesc = f16_idesc(kBM, kBN);
 
 // ---------------------------------------------------------------- arguments
 // Work is split into units (KV head h, 128-row block rb, column segment seg):
@@ -314,7 +241,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const uint32_t kb = (uint32_t)k * 32u;     // 16 bf16 of K per MMA
                         const uint32_t atom = kb / rb, within = kb % rb;
                         tc_mma(d, umma_desc(Asa + atom * kBM * rb + within, rb),
-                               umma_desc(Bs + atom * kBN * rb + within, rb), k > 0 ? 1u : 0u);
+                               umma_desc(Bs + atom * kBN * rb + within, rb), kIdesc, k > 0 ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
                     tc_commit(&tfull[acc]);

@@ -160,3 +160,18 @@ def make_prefill_inputs(w: Workload, seed: int | None = None) -> dict[str, torch
     k = _normal_bf16((w.T, w.hkv, w.d), gen)
     v = _normal_bf16((w.T, w.hkv, w.d), gen)
     return {"q": q, "qt": qt, "k": k, "v": v, "kt": kt, "q_start": w.T - w.nq}
+
+
+def make_projection_inputs(seed: int, batch: int, T: int, H: int, d: int, r: int, nbases: int,
+                           x_range: int | None = 3, p_range: int | None = 2) -> dict[str, torch.Tensor]:
+    """Host bf16 tensors for scoring preparation: rows x [batch, T, H, d] and
+    bases P [nbases, r, d]. Integer-valued when a range is given (uniform in
+    [-R, R]), else x ~ N(0, 1) and P ~ N(0, 1) / sqrt(d) (an approximately
+    orthonormal random basis). Draw order: x, P."""
+    gen = torch.Generator().manual_seed(seed)
+    x = _int_bf16((batch, T, H, d), x_range, gen) if x_range is not None else _normal_bf16((batch, T, H, d), gen)
+    if p_range is not None:
+        P = _int_bf16((nbases, r, d), p_range, gen)
+    else:
+        P = (_normal_bf16((nbases, r, d), gen).to(torch.float32) / math.sqrt(d)).to(torch.bfloat16)
+    return {"x": x, "P": P}

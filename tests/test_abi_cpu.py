@@ -142,3 +142,40 @@ def test_fp8_validation():
     assert lib.lsa_score_fp8(ctypes.byref(d), ALIGNED, MISALIGNED, ALIGNED, None) == -2
     assert lib.lsa_decode_step_fp8(ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 16, f(0.1),
                                    None, ALIGNED, ALIGNED, 16, None) == -4
+
+
+def _pd(**kw):
+    base = dict(batch=2, T=1000, H=8, d=128, r=64, nbases=8)
+    base.update(kw)
+    return L.lsa_proj_dims(*(base[k] for k in ("batch", "T", "H", "d", "r", "nbases")))
+
+
+@pytest.mark.parametrize("fn", ["lsa_project", "lsa_project_fp8"])
+def test_project_validation(fn):
+    """Every rejection happens on the host, before any device use."""
+    f = getattr(L.lib(), fn)
+    ok = _pd()
+    call = lambda d, x=ALIGNED, P=ALIGNED, t0=0, n=10, y=ALIGNED, st=None: f(  # noqa: E731
+        ctypes.byref(d), x, P, t0, n, y, st, None)
+    assert call(ok, x=None) == -1
+    assert call(ok, y=None) == -1
+    assert call(_pd(H=6, nbases=4)) == -1            # H % nbases != 0
+    assert call(_pd(T=0)) == -1
+    assert call(ok, t0=-1) == -3
+    assert call(ok, t0=995, n=6) == -3               # t0 + n > T
+    assert call(ok, n=-1) == -3
+    assert call(ok, x=MISALIGNED) == -2
+    assert call(ok, st=ctypes.c_void_p(ALIGNED.value + 2)) == -2
+    for kw in (dict(d=48), dict(d=24), dict(d=320), dict(r=8), dict(r=40), dict(r=144), dict(d=256, r=96)):
+        assert call(_pd(**kw)) == -7, kw
+    assert call(ok, n=0) == 0                        # nothing to do, nothing launched
+
+
+def test_update_centroids_validation():
+    lib = L.lib()
+    d = _dims()
+    assert lib.lsa_update_centroids(ctypes.byref(d), None, 64, 0, 1, ALIGNED, None) == -1
+    assert lib.lsa_update_centroids(ctypes.byref(d), ALIGNED, 0, 0, 1, ALIGNED, None) == -1
+    assert lib.lsa_update_centroids(ctypes.byref(d), ALIGNED, 64, d.T, 1, ALIGNED, None) == -3
+    assert lib.lsa_update_centroids(ctypes.byref(d), ALIGNED, 64, 0, 1, MISALIGNED, None) == -2
+    assert lib.lsa_update_centroids(ctypes.byref(d), ALIGNED, 64, 5, 0, ALIGNED, None) == 0
