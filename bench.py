@@ -864,8 +864,10 @@ def cpu_prepare_sample(x, P, budget_s=12.0, max_tokens=None):
     t0 = time.perf_counter()
     n = 0
     chunk = 256
+    T = x.shape[1]
     while True:
-        xs = x[0, n:n + chunk].to(torch_float32()).numpy()
+        s0 = n % T
+        xs = x[0, s0:min(T, s0 + chunk)].to(torch_float32()).numpy()
         O.project_bf16(xs, Pn, 1)
         n += xs.shape[0]
         el = time.perf_counter() - t0
