@@ -38,6 +38,8 @@ if ROOT not in sys.path:
 
 METRIC = "sparse decode steps/s per layer at 128K, B=2048; achieved HBM GB/s vs peak"
 METRIC_FP8 = "sparse decode steps/s per layer at 128K, B=2048, FP8 (E4M3) projected-key cache; HBM GB/s vs peak"
+METRIC_PAGED = ("sparse decode steps/s per layer at 128K, B=2048, paged KV cache (page size 1, slots in random "
+                "order); HBM GB/s vs peak")
 UNIT = "steps/s"
 WORKLOAD = "decode_128k"
 FALLBACK_HBM_GBS = 6650.0
@@ -312,7 +314,8 @@ def run_reference(args, rank, world):
     step_s = unit_s * w.batch * w.hkv
     value = 1.0 / step_s
     line = {
-        "impl": "reference", "metric": METRIC_FP8 if args.workload == "decode_128k_fp8" else METRIC,
+        "impl": "reference",
+        "metric": {"decode_128k_fp8": METRIC_FP8, "decode_128k_paged": METRIC_PAGED}.get(args.workload, METRIC),
         "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -337,11 +340,20 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     lsa.lib()
     fp8 = args.workload == "decode_128k_fp8"
+    paged = args.workload == "decode_128k_paged"
     w = I.workload(WORKLOAD)
     x = I.make_decode_inputs(w, seed=rank_seed(w, rank))
     d = {k: x[k].to(dev) for k in ("q", "qt", "k", "v", "kt")}
     if fp8:   # the same integer values, stored as E4M3 (exact)
         d["kt8"] = d["kt"].to(torch.float8_e4m3fn)
+    if paged:   # the same K/V rows in pools, token (b, t) at a random slot
+        nslots = w.batch * w.T
+        perm = torch.randperm(nslots, generator=torch.Generator().manual_seed(w.seed + 17)).to(dev)
+        d["page_table"] = perm.to(torch.int32).view(w.batch, w.T)
+        for name in ("k", "v"):
+            pool = torch.empty((nslots, w.hkv, w.d), dtype=torch.bfloat16, device=dev)
+            pool[perm] = d[name].view(nslots, w.hkv, w.d)
+            d[name + "_pool"] = pool
     dims = _lib.decode_dims(d["q"], d["qt"], d["k"])
     ws = lsa.workspace(dims, w.B, device=dev)
     idx = torch.empty((w.batch, w.hkv, w.B), dtype=torch.int32, device=dev)
@@ -351,6 +363,9 @@ def run_ours(args, rank, world, local_rank):
     def step():
         if fp8:
             lsa.lsa_decode_step_fp8(d["q"], d["qt"], d["k"], d["v"], d["kt8"], w.B, idx_out=idx, out=out, ws=ws)
+        elif paged:
+            lsa.lsa_decode_step_paged(d["q"], d["qt"], d["k_pool"], d["v_pool"], d["page_table"], d["kt"], w.B,
+                                      idx_out=idx, out=out, ws=ws)
         else:
             lsa.lsa_decode_step(d["q"], d["qt"], d["k"], d["v"], d["kt"], w.B, idx_out=idx, out=out, ws=ws)
 
@@ -401,12 +416,19 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     lsa.lsa_score(d["qt"], d["kt"], scores)
     lsa.lsa_topk(scores, w.B, idx)
-    lsa.lsa_indexed_attn(d["q"], d["k"], d["v"], idx, out=out, ws=ws)
     reps = 8
+
+    def attn_call():
+        if paged:
+            lsa.lsa_indexed_attn_paged(d["q"], d["k_pool"], d["v_pool"], d["page_table"], idx, out=out, ws=ws)
+        else:
+            lsa.lsa_indexed_attn(d["q"], d["k"], d["v"], idx, out=out, ws=ws)
+
+    attn_call()
 
     def attn_after_flush():
         flush.zero_()
-        lsa.lsa_indexed_attn(d["q"], d["k"], d["v"], idx, out=out, ws=ws)
+        attn_call()
 
     score_call = (lambda: lsa.lsa_score_fp8(d["qt"], d["kt8"], scores)) if fp8 else \
         (lambda: lsa.lsa_score(d["qt"], d["kt"], scores))
@@ -476,12 +498,16 @@ def run_ours(args, rank, world, local_rank):
             cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                    "sample": f"{n} (sequence, KV head) units of the 128K workload ({el:.1f} s), scaled to steps"}
         line = {
-            "metric": METRIC_FP8 if fp8 else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps,
+            "metric": METRIC_FP8 if fp8 else (METRIC_PAGED if paged else METRIC), "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_dict(w, {"parallelism": f"replicas{world}" if world > 1 else "single",
-                                      **({"workload": "decode_128k_fp8", "kt_dtype": "fp8_e4m3"} if fp8 else {})}),
+                                      **({"workload": "decode_128k_fp8", "kt_dtype": "fp8_e4m3"} if fp8 else {}),
+                                      **({"workload": "decode_128k_paged",
+                                          "kv_layout": "pools [batch*T, hkv, d] bf16, page size 1, page table "
+                                                       "[batch, T] int32 (a random permutation of the slots)"}
+                                         if paged else {})}),
             "roofline": {"bound": "hbm", "kernel": "score_q64_kernel (lsa_score_fp8)" if fp8 else
                          "score_q64_kernel (lsa_score)", "achieved": achieved, "peak": peak,
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
@@ -1054,11 +1080,12 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["decode_128k", "decode_128k_fp8", "prefill_128k", "llama8b_32k",
-                                           "hier_1m", "prepare_128k"],
+    ap.add_argument("--workload", choices=["decode_128k", "decode_128k_fp8", "decode_128k_paged", "prefill_128k",
+                                           "llama8b_32k", "hier_1m", "prepare_128k"],
                     default="decode_128k",
                     help="decode_128k (the headline), decode_128k_fp8 (the same step over an FP8 projected-key "
-                         "cache), prefill_128k (indexer + indexed attention), the L2-resident decode steps "
+                         "cache), decode_128k_paged (the same step with K/V in page-size-1 pools), prefill_128k "
+                         "(indexer + indexed attention), the L2-resident decode steps "
                          "llama8b_32k and hier_1m, or prepare_128k (scoring preparation: projecting the 128K "
                          "key cache, and the decode-time append)")
     ap.add_argument("--ncu-case", choices=["score", "score8", "topk", "attn", "step", "project"], default=None,

@@ -210,6 +210,34 @@ LSA_API lsa_status lsa_decode_step_fp8(const lsa_dims* dims, const lsa_bf16* q, 
 LSA_API lsa_status lsa_block_centroids(const lsa_dims* dims, const lsa_bf16* kt, int blk,
                                lsa_bf16* centroids, void* stream);
 
+/* ---- Paged KV cache, page size 1 ("Their 42x decode speedup never compiled
+ * on my GPU", What their numbers claim: the release's serving configurations
+ * pin a KV page size of 1, one token per page, which token-level index sets
+ * need). K and V live in pools k_pool / v_pool [nslots, hkv, d] bf16, and
+ * page_table [batch, T] int32 gives the pool slot of logical position t of
+ * sequence b. The index sets stay logical positions; attention reads row
+ * (page_table[b, t], h) of the pools in place. A slot outside [0, nslots)
+ * for a selected position is skipped and sets LSA_DEV_BAD_INDEX. The
+ * projected-key cache kt stays contiguous [batch, T, hkv, r]. nslots >= 1,
+ * page_table 16-byte aligned. Workspace: lsa_workspace_size(dims, B, 0, 0). */
+LSA_API lsa_status lsa_indexed_attn_paged(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* k_pool,
+                                          const lsa_bf16* v_pool, int nslots, const int32_t* page_table,
+                                          const int32_t* idx, int B, float scale, lsa_bf16* out, void* ws,
+                                          size_t ws_bytes, void* stream);
+
+/* lsa_decode_step (flat scoring) with the KV cache in paged pools. */
+LSA_API lsa_status lsa_decode_step_paged(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* qt,
+                                         const lsa_bf16* k_pool, const lsa_bf16* v_pool, int nslots,
+                                         const int32_t* page_table, const lsa_bf16* kt, int B, float scale,
+                                         int32_t* idx_out, lsa_bf16* out, void* ws, size_t ws_bytes,
+                                         void* stream);
+
+/* Cross-layer index reuse (LongCat Sparse Attention, Abstract, strategy (2)
+ * Cross-Layer Indexing: one layer's index sets serve the consecutive layers)
+ * needs no entry of its own: pass the idx that lsa_decode_step (idx_out) or
+ * lsa_topk produced for one layer to lsa_indexed_attn / lsa_indexed_attn_paged
+ * with the next layers' q, k and v. */
+
 /* ---- Scoring preparation (JSSA, Fig. 9: the key projection that fills the
  * projected-key cache; Fig. 1: keys and the group's queries are scored in a
  * shared low-dimensional subspace). Every basis P[j] holds r vectors of length

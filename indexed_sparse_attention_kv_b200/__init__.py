@@ -16,6 +16,8 @@ from ._lib import (  # noqa: F401
     lsa_dims,
     lsa_indexed_attn,
     lsa_indexed_attn_noalloc,
+    lsa_indexed_attn_paged,
+    lsa_decode_step_paged,
     lsa_prefill_attn,
     lsa_prefill_index,
     lsa_prefill_workspace_size,

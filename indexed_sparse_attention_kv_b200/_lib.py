@@ -67,6 +67,8 @@ _SIGS = {
     "lsa_decode_step_fp8": (_I, [_DIMS, _P, _P, _P, _P, _P, _I, ctypes.c_float, _P, _P, _P, _SZ, _P]),
     "lsa_decode_step": (_I, [_DIMS, _P, _P, _P, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _P, _SZ, _P]),
     "lsa_block_centroids": (_I, [_DIMS, _P, _I, _P, _P]),
+    "lsa_indexed_attn_paged": (_I, [_DIMS, _P, _P, _P, _I, _P, _P, _I, ctypes.c_float, _P, _P, _SZ, _P]),
+    "lsa_decode_step_paged": (_I, [_DIMS, _P, _P, _P, _P, _I, _P, _P, _I, ctypes.c_float, _P, _P, _P, _SZ, _P]),
     "lsa_project": (_I, [ctypes.POINTER(lsa_proj_dims), _P, _P, _I, _I, _P, _P, _P]),
     "lsa_project_fp8": (_I, [ctypes.POINTER(lsa_proj_dims), _P, _P, _I, _I, _P, _P, _P]),
     "lsa_update_centroids": (_I, [_DIMS, _P, _I, _I, _I, _P, _P]),
@@ -248,6 +250,59 @@ def lsa_decode_step(q, qt, k, v, kt, B: int, scale: float | None = None, centroi
         ws = workspace(dims, B, blk, keep, device=q.device)
     _check("lsa_decode_step", lib().lsa_decode_step(
         ctypes.byref(dims), _ptr(q), _ptr(qt), _ptr(k), _ptr(v), _ptr(kt), _ptr(centroids), int(blk), int(keep),
+        int(B), ctypes.c_float(scale), _ptr(idx_out), _ptr(out), _ptr(ws), ws.numel(), _stream(q)))
+    return idx_out, out
+
+
+def _paged_dims(q, k_pool, page_table, r):
+    batch, hq, d = q.shape
+    nslots, hkv, _ = k_pool.shape
+    T = page_table.shape[1]
+    return make_dims(batch, hq, hkv, d, r, T), nslots
+
+
+def lsa_indexed_attn_paged(q, k_pool, v_pool, page_table, idx, scale: float | None = None, out=None,
+                           ws=None) -> torch.Tensor:
+    """Indexed attention over a paged KV cache (lsa.h: lsa_indexed_attn_paged): k_pool / v_pool
+    [nslots, hkv, d], page_table [batch, T] int32 (pool slot of each logical position), idx
+    [batch, hkv, B] logical positions."""
+    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool")):
+        _cuda(t, n, torch.bfloat16)
+    _cuda(page_table, "page_table", torch.int32)
+    _cuda(idx, "idx", torch.int32)
+    dims, nslots = _paged_dims(q, k_pool, page_table, 16)
+    B = idx.shape[-1]
+    scale = 1.0 / math.sqrt(dims.d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    _cuda(out, "out", torch.bfloat16)
+    if ws is None:
+        ws = workspace(dims, B, device=q.device)
+    _check("lsa_indexed_attn_paged", lib().lsa_indexed_attn_paged(
+        ctypes.byref(dims), _ptr(q), _ptr(k_pool), _ptr(v_pool), int(nslots), _ptr(page_table), _ptr(idx), int(B),
+        ctypes.c_float(scale), _ptr(out), _ptr(ws), ws.numel(), _stream(q)))
+    return out
+
+
+def lsa_decode_step_paged(q, qt, k_pool, v_pool, page_table, kt, B: int, scale: float | None = None, idx_out=None,
+                          out=None, ws=None, return_idx: bool = True):
+    """One flat decode step over a paged KV cache (lsa.h: lsa_decode_step_paged); kt [batch, T, hkv, r]
+    stays contiguous. Returns (idx [batch, hkv, B] or None, out [batch, hq, d])."""
+    for t, n in ((q, "q"), (qt, "qt"), (k_pool, "k_pool"), (v_pool, "v_pool"), (kt, "kt")):
+        _cuda(t, n, torch.bfloat16)
+    _cuda(page_table, "page_table", torch.int32)
+    dims, nslots = _paged_dims(q, k_pool, page_table, kt.shape[-1])
+    scale = 1.0 / math.sqrt(dims.d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if idx_out is None and return_idx:
+        idx_out = torch.empty((dims.batch, dims.hkv, B), dtype=torch.int32, device=q.device)
+    if idx_out is not None:
+        _cuda(idx_out, "idx_out", torch.int32)
+    if ws is None:
+        ws = workspace(dims, B, device=q.device)
+    _check("lsa_decode_step_paged", lib().lsa_decode_step_paged(
+        ctypes.byref(dims), _ptr(q), _ptr(qt), _ptr(k_pool), _ptr(v_pool), int(nslots), _ptr(page_table), _ptr(kt),
         int(B), ctypes.c_float(scale), _ptr(idx_out), _ptr(out), _ptr(ws), ws.numel(), _stream(q)))
     return idx_out, out
 

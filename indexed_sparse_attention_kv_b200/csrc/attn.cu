@@ -51,7 +51,9 @@ struct AttnArgs {
     float* pl;
     float* po;                // [units, smax, G, D]
     unsigned* counters;       // [units] finished-segment counters (zero between launches)
-    long long kv_bstride_rows;   // T * hkv for decode, 0 for prefill (one shared cache)
+    long long kv_bstride_rows;   // T * hkv for decode, 0 for prefill (one shared cache) and paged pools
+    const int32_t* slots;        // optional page table (page size 1): [nb, T] pool row of position t
+    long long nslots;            // rows of the K/V pools when paged
     int hq, hkv, T, B;
     int units, tiles_per_unit, ctas, smax;
     long long total_tiles;
@@ -151,6 +153,15 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
         if (t < -1 || t >= a.T) {
             set_status(a.status, kStatusBadIndex);
             t = -1;
+        }
+        if (a.slots && t >= 0) {   // logical position -> pool row
+            const int p = __ldg(a.slots + (size_t)(u / a.hkv) * a.T + t);
+            if (p < 0 || p >= a.nslots) {
+                set_status(a.status, kStatusBadIndex);
+                t = -1;
+            } else {
+                t = p;
+            }
         }
         return t;
     };
@@ -545,8 +556,11 @@ AttnPlan plan_attn(int nb, int hkv, int G, int B, int d, int num_sms) {
 cudaError_t launch_attn(const LaunchCtx& ctx, const AttnPlan& plan, const uint16_t* q, const uint16_t* k,
                         const uint16_t* v, const int32_t* idx, int B, float scale, uint16_t* out, float* pm, float* pl,
                         float* po, unsigned* counters, int nb, int hq, int hkv, int d, int T,
-                        long long kv_bstride_rows, unsigned* status) {
+                        long long kv_bstride_rows, unsigned* status, const int32_t* slots, long long nslots) {
     AttnArgs a{};
+    a.slots = slots;
+    a.nslots = nslots;
+    if (slots) kv_bstride_rows = 0;
     a.q = q;
     a.k = reinterpret_cast<const uint8_t*>(k);
     a.v = reinterpret_cast<const uint8_t*>(v);

@@ -353,6 +353,58 @@ lsa_status lsa_decode_step(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf
     return from_cuda(e);
 }
 
+lsa_status lsa_indexed_attn_paged(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* k_pool,
+                                  const lsa_bf16* v_pool, int nslots, const int32_t* page_table, const int32_t* idx,
+                                  int B, float scale, lsa_bf16* out, void* ws, size_t ws_bytes, void* stream) {
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if ((s = check_B(B)) != LSA_OK) return s;
+    if (!q || !k_pool || !v_pool || !page_table || !idx || !out || nslots < 1) return LSA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(page_table) || !aligned16(idx) ||
+        !aligned16(out))
+        return LSA_ERR_ALIGN;
+    if (!std::isfinite(scale)) return LSA_ERR_ARG;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    const DecodeLayout L = decode_layout(dims, B, 0, 0, ctx.num_sms);
+    if ((s = check_ws(ws, ws_bytes, L.total)) != LSA_OK) return s;
+    return from_cuda(lsa::launch_attn(ctx, L.plan, q, k_pool, v_pool, idx, B, scale, out, at<float>(ws, L.pm),
+                                      at<float>(ws, L.pl), at<float>(ws, L.po), at<unsigned>(ws, L.counters),
+                                      dims->batch, dims->hq, dims->hkv, dims->d, dims->T, 0,
+                                      at<unsigned>(ws, L.status), page_table, nslots));
+}
+
+lsa_status lsa_decode_step_paged(const lsa_dims* dims, const lsa_bf16* q, const lsa_bf16* qt, const lsa_bf16* k_pool,
+                                 const lsa_bf16* v_pool, int nslots, const int32_t* page_table, const lsa_bf16* kt,
+                                 int B, float scale, int32_t* idx_out, lsa_bf16* out, void* ws, size_t ws_bytes,
+                                 void* stream) {
+    lsa_status s = check_dims(dims);
+    if (s != LSA_OK) return s;
+    if ((s = check_B(B)) != LSA_OK) return s;
+    if (!q || !qt || !k_pool || !v_pool || !page_table || !kt || !out || nslots < 1) return LSA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(qt) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(page_table) ||
+        !aligned16(kt) || !aligned16(out))
+        return LSA_ERR_ALIGN;
+    if (idx_out && !aligned16(idx_out)) return LSA_ERR_ALIGN;
+    if (!std::isfinite(scale)) return LSA_ERR_ARG;
+    const lsa::LaunchCtx ctx = make_ctx(stream);
+    const DecodeLayout L = decode_layout(dims, B, 0, 0, ctx.num_sms);
+    if ((s = check_ws(ws, ws_bytes, L.total)) != LSA_OK) return s;
+    unsigned* status = at<unsigned>(ws, L.status);
+    int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
+    bool hist = false;
+    uint32_t* gh = at<uint32_t>(ws, L.hist);
+    cudaError_t e = lsa::launch_score(ctx, qt, kt, at<float>(ws, L.scores), dims->batch, dims->hq, dims->hkv, dims->r,
+                                      dims->T, 0, status, gh, &hist);
+    if (e == cudaSuccess)
+        e = lsa::launch_topk(ctx, at<float>(ws, L.scores), dims->batch * dims->hkv, dims->T, B, idx, nullptr, 0, 0,
+                             hist ? gh : nullptr);
+    if (e == cudaSuccess)
+        e = lsa::launch_attn(ctx, L.plan, q, k_pool, v_pool, idx, B, scale, out, at<float>(ws, L.pm),
+                             at<float>(ws, L.pl), at<float>(ws, L.po), at<unsigned>(ws, L.counters), dims->batch,
+                             dims->hq, dims->hkv, dims->d, dims->T, 0, status, page_table, nslots);
+    return from_cuda(e);
+}
+
 static bool fp8_shape_ok(const lsa_dims* d) {
     return d->r == 64 && (d->hkv == 4 || d->hkv == 8 || d->hkv == 16 || d->hkv == 32);
 }

@@ -110,11 +110,14 @@ cudaError_t launch_centroid_update(const LaunchCtx& ctx, const uint16_t* kt, uin
 AttnPlan plan_attn(int nb, int hkv, int G, int B, int d, int num_sms);
 
 // pm/pl: [units, smax, G] fp32, po: [units, smax, G, d] fp32, counters:
-// [units] uint32, zero on entry and left zero.
+// [units] uint32, zero on entry and left zero. slots (optional): page table
+// [nb, T] of pool rows (k/v then [nslots, hkv, d]); entries outside
+// [0, nslots) are skipped and flag LSA_DEV_BAD_INDEX.
 cudaError_t launch_attn(const LaunchCtx& ctx, const AttnPlan& plan, const uint16_t* q, const uint16_t* k,
                         const uint16_t* v, const int32_t* idx, int B, float scale, uint16_t* out, float* pm, float* pl,
                         float* po, unsigned* counters, int nb, int hq, int hkv, int d, int T,
-                        long long kv_bstride_rows, unsigned* status);
+                        long long kv_bstride_rows, unsigned* status, const int32_t* slots = nullptr,
+                        long long nslots = 0);
 
 // Prefill indexer plan: sample stride, selection constants and the byte
 // offsets of its buffers inside the caller's workspace region.

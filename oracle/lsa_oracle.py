@@ -60,6 +60,8 @@ __all__ = [
     "prefill_scores",
     "prefill_index",
     "prefill_attention",
+    "paged_rows",
+    "indexed_attention_paged",
     "round_to_bf16",
     "round_to_e4m3",
     "project_rows",
@@ -260,6 +262,26 @@ def prefill_attention(q_rows, k, v, idx, scale: float) -> np.ndarray:
     """Indexed attention for every prefill query row: out [n, hq, d]."""
     q_rows = _f64(q_rows)
     return np.stack([indexed_attention(q_rows[i], k, v, idx[i], scale) for i in range(q_rows.shape[0])])
+
+
+def paged_rows(pool, slots) -> np.ndarray:
+    """The logical [T, hkv, d] cache of one sequence held in a pool of slots
+    (page size 1: "Their 42x decode speedup never compiled on my GPU", What
+    their numbers claim): row t is pool[slots[t]]; a slot outside the pool
+    (e.g. -1, an unfilled position) gives a NaN row, which a correct index set
+    never selects."""
+    pool = _f64(pool)
+    slots = np.asarray(slots)
+    out = np.full((len(slots),) + pool.shape[1:], np.nan)
+    ok = (slots >= 0) & (slots < pool.shape[0])
+    out[ok] = pool[slots[ok]]
+    return out
+
+
+def indexed_attention_paged(q, k_pool, v_pool, slots, idx, scale: float) -> np.ndarray:
+    """indexed_attention over the K/V rows of a paged cache: the index sets
+    hold logical positions, mapped through ``slots`` [T] to pool rows."""
+    return indexed_attention(q, paged_rows(k_pool, slots), paged_rows(v_pool, slots), idx, scale)
 
 
 def default_scale(d: int) -> float:

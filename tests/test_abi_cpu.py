@@ -179,3 +179,24 @@ def test_update_centroids_validation():
     assert lib.lsa_update_centroids(ctypes.byref(d), ALIGNED, 64, d.T, 1, ALIGNED, None) == -3
     assert lib.lsa_update_centroids(ctypes.byref(d), ALIGNED, 64, 0, 1, MISALIGNED, None) == -2
     assert lib.lsa_update_centroids(ctypes.byref(d), ALIGNED, 64, 5, 0, ALIGNED, None) == 0
+
+
+def test_paged_validation():
+    lib = L.lib()
+    f = ctypes.c_float
+    d = _dims()
+    a = lambda **kw: lib.lsa_indexed_attn_paged(  # noqa: E731
+        ctypes.byref(d), kw.get("q", ALIGNED), ALIGNED, ALIGNED, kw.get("nslots", 10), kw.get("pt", ALIGNED),
+        ALIGNED, 16, f(0.1), ALIGNED, kw.get("ws", ALIGNED), kw.get("wsb", 1 << 40), None)
+    assert a(q=None) == -1
+    assert a(pt=None) == -1
+    assert a(nslots=0) == -1
+    assert a(pt=MISALIGNED) == -2
+    assert a(wsb=16) == -4
+    s = lambda **kw: lib.lsa_decode_step_paged(  # noqa: E731
+        ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, ALIGNED, kw.get("nslots", 10), kw.get("pt", ALIGNED),
+        kw.get("kt", ALIGNED), 16, f(0.1), None, ALIGNED, ALIGNED, kw.get("wsb", 1 << 40), None)
+    assert s(kt=None) == -1
+    assert s(nslots=-3) == -1
+    assert s(pt=MISALIGNED) == -2
+    assert s(wsb=16) == -4

@@ -290,6 +290,31 @@ def check_golden(o):
 
 # ------------------------------------------------------------------ scoring preparation
 
+def check_paged_attention(o):
+    """Identity page table == the contiguous cache; a permuted pool read
+    through the matching table == the contiguous cache; unfilled slots of
+    positions outside the index sets do not matter."""
+    rng = np.random.default_rng(27)
+    T, hkv, hq, d, B = 40, 2, 4, 8, 6
+    q = rng.standard_normal((hq, d))
+    k = rng.standard_normal((T, hkv, d))
+    v = rng.standard_normal((T, hkv, d))
+    idx = np.stack([np.sort(rng.choice(T, B, replace=False)) for _ in range(hkv)])
+    ref = o.indexed_attention(q, k, v, idx, 0.3)
+    assert np.array_equal(o.indexed_attention_paged(q, k, v, np.arange(T), idx, 0.3), ref)
+    perm = rng.permutation(T + 5)                     # pool with 5 spare slots
+    pool_k = rng.standard_normal((T + 5, hkv, d))
+    pool_v = rng.standard_normal((T + 5, hkv, d))
+    slots = perm[:T]
+    pool_k[slots] = k
+    pool_v[slots] = v
+    assert np.allclose(o.indexed_attention_paged(q, pool_k, pool_v, slots, idx, 0.3), ref, rtol=0, atol=1e-12)
+    holes = slots.copy()
+    unused = np.setdiff1d(np.arange(T), idx.ravel())
+    holes[unused[:3]] = -1
+    assert np.allclose(o.indexed_attention_paged(q, pool_k, pool_v, holes, idx, 0.3), ref, rtol=0, atol=1e-12)
+
+
 def check_round_bf16(o):
     """fp32-representable values: one rounding, so torch's fp32 -> bf16 cast
     (round to nearest even) is the reference; plus hand-derived ties."""
@@ -388,7 +413,7 @@ CHECKS = [
     check_attention_unselected_irrelevant, check_centroids_closed_form, check_hier_reductions,
     check_prefill_vs_decode_prefix, check_golden,
     check_round_bf16, check_round_e4m3, check_project_shifted_unit_basis, check_project_orthonormal,
-    check_project_integer_exact, check_update_centroids,
+    check_project_integer_exact, check_update_centroids, check_paged_attention,
 ]
 
 
@@ -583,7 +608,14 @@ def _cent_wrong_block(c, kt, t0, n, blk):  # token t lands in block (t + 1) // b
     return c
 
 
+def _paged_inverse(q, k_pool, v_pool, slots, idx, scale):   # reads the table backwards (slot -> position)
+    slots = np.asarray(slots)
+    inv = np.argsort(np.where(slots >= 0, slots, np.iinfo(np.int64).max))[: len(slots)]
+    return O.indexed_attention(q, O.paged_rows(k_pool, inv), O.paged_rows(v_pool, inv), idx, scale)
+
+
 MUTANTS = {
+    "paged_table_inverted": dict(indexed_attention_paged=_paged_inverse),
     "bf16_truncates": dict(round_to_bf16=_bf16_truncate),
     "bf16_ties_away": dict(round_to_bf16=_bf16_ties_away),
     "e4m3_not_saturated": dict(round_to_e4m3=_e4m3_no_saturation),
