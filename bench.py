@@ -113,6 +113,23 @@ def source_hash(paths):
     return h.hexdigest()[:16]
 
 
+PROJECT_SOURCES = ["indexed_sparse_attention_kv_b200/csrc/project.cu", "indexed_sparse_attention_kv_b200/csrc/tcgen05.cuh",
+                   "indexed_sparse_attention_kv_b200/csrc/lsa_common.cuh"]
+
+
+def project_traffic():
+    """DRAM bytes per projection launch (prepare_128k) from the committed ncu
+    summary, or None if the kernel's sources changed since it was captured."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic_project.json")) as f:
+            t = json.load(f)
+        if t.get("source_hash") != source_hash(PROJECT_SOURCES):
+            return None
+        return float(t["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
 def scorer_traffic(w):
     """DRAM bytes per scorer launch from the committed ncu summary, or None if
     the scorer's sources changed since it was captured."""
@@ -1014,7 +1031,7 @@ def run_prepare(args, rank, world, local_rank):
             "config": {"workload": "prepare_128k", **sh, "nbases": sh["H"],
                        "l2": "inputs exceed L2 (1 GiB of keys per step)"},
             "roofline": {"bound": "hbm", "kernel": "project_kernel (lsa_project)", "achieved": achieved,
-                         "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": project_traffic(),
                          "peak_kind": peak_kind, "algorithmic_bytes_per_launch": byt, "avg_launch_ms": per_ms},
             "append_us": append_us,
             "cpu_baseline": cpu,
