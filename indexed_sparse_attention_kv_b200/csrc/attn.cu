@@ -119,7 +119,7 @@ struct AttnLayout {
     static constexpr int kTotal = kStages * kStage + kFixed;
 };
 
-template <int D, int G>
+template <int D, int G, bool PAGED>
 __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
     using Lay = AttnLayout<D, G>;
     constexpr int S = Lay::kStages;
@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
             set_status(a.status, kStatusBadIndex);
             t = -1;
         }
-        if (a.slots && t >= 0) {   // logical position -> pool row
+        if (PAGED && t >= 0) {   // logical position -> pool row
             const int p = __ldg(a.slots + (size_t)(u / a.hkv) * a.T + t);
             if (p < 0 || p >= a.nslots) {
                 set_status(a.status, kStatusBadIndex);
@@ -491,7 +491,7 @@ template <int D, int G>
 cudaError_t launch_attn_t(const LaunchCtx& ctx, AttnArgs a) {
     using Lay = AttnLayout<D, G>;
     const size_t smem = Lay::kTotal;
-    auto kern = attn_kernel<D, G>;
+    auto kern = a.slots ? attn_kernel<D, G, true> : attn_kernel<D, G, false>;
     cudaError_t e = ensure_dyn_smem((const void*)kern, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
