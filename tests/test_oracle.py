@@ -274,6 +274,15 @@ def check_golden(o):
     out = o.indexed_attention(q, k, v, np.array(g["idx"]), g["scale"])
     assert np.allclose(out, g["out"], rtol=0, atol=1e-14)
 
+    g = _load("scoring_preparation.json")
+    x, P = np.array(g["x"], dtype=np.float64), np.array(g["P"], dtype=np.float64)
+    assert np.array_equal(o.project_rows(x, P, g["G"]), np.array(g["exact"], dtype=np.float64))
+    assert np.array_equal(o.round_to_bf16(o.project_rows(x, P, g["G"])), np.array(g["bf16"], dtype=np.float64))
+    assert np.array_equal(o.round_to_e4m3(o.project_rows(x, P, g["G"])), np.array(g["e4m3"], dtype=np.float64))
+    c = o.update_centroids(np.array(g["centroid_start"], dtype=np.float64), np.array(g["kt"], dtype=np.float64),
+                           g["t0"], g["n"], g["blk"])
+    assert np.array_equal(c, np.array(g["centroid_end"], dtype=np.float64))
+
     g = _load("hierarchical_blocks.json")
     kt = np.array(g["kt"], dtype=np.float64)
     assert np.array_equal(o.block_centroids(kt, g["blk"]), np.array(g["centroids"], dtype=np.float64))
