@@ -56,10 +56,11 @@ def test_paged_step_equals_contiguous_and_oracle(case):
     idx0, out0 = lsa.lsa_decode_step(d["q"], d["qt"], d["k"], d["v"], d["kt"], w.B)
     idx1, out1 = lsa.lsa_decode_step_paged(d["q"], d["qt"], kp.cuda(), vp.cuda(), table.cuda(), d["kt"], w.B)
     out2 = lsa.lsa_indexed_attn_paged(d["q"], kp.cuda(), vp.cuda(), table.cuda(), idx0)
+    out3 = lsa.lsa_indexed_attn(d["q"], d["k"], d["v"], idx0)
     torch.cuda.synchronize()
     assert torch.equal(idx1, idx0)
-    assert torch.equal(out1, out0)
-    assert torch.equal(out2, out0)
+    assert torch.equal(out1, out0)     # the same step over the same rows
+    assert torch.equal(out2, out3)     # the same attention kernel over the same rows
     ref_idx, _ = oracle_decode(x, w)
     assert np.array_equal(idx1.cpu().numpy(), ref_idx)
     for b in range(w.batch):
