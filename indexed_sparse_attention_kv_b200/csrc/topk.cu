@@ -44,7 +44,7 @@ constexpr int kListPerWarp = 128;                       // (key, position) entri
 constexpr int kListCap = kListPerWarp * kTopkWarps;     // per CTA
 constexpr int kGatherCap = 4096;                        // bin-b0 keys of the whole cluster
 constexpr int kMaxCluster = 8;
-constexpr int kBatch = 8;                               // 128-key steps whose loads are issued together
+constexpr int kBatch = 2;                               // 128-key steps whose loads are issued together
 
 struct TopkArgs {
     const float* scores;      // [rows, n]
