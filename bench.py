@@ -901,16 +901,18 @@ def prepare_bytes(sh):
 def cpu_prepare_sample(x, P, budget_s=12.0, max_tokens=None):
     """Oracle projection of whole token rows (all heads) of sequence 0 until the
     budget (or max_tokens) is spent; returns (GB/s of the algorithmic bytes, tokens, seconds)."""
+    import torch
+
     import oracle.lsa_oracle as O
 
-    Pn = P.to(torch_float32()).numpy()
+    Pn = P.to(torch.float32).numpy()
     t0 = time.perf_counter()
     n = 0
     chunk = 256
     T = x.shape[1]
     while True:
         s0 = n % T
-        xs = x[0, s0:min(T, s0 + chunk)].to(torch_float32()).numpy()
+        xs = x[0, s0:min(T, s0 + chunk)].to(torch.float32).numpy()
         O.project_bf16(xs, Pn, 1)
         n += xs.shape[0]
         el = time.perf_counter() - t0
@@ -919,11 +921,6 @@ def cpu_prepare_sample(x, P, budget_s=12.0, max_tokens=None):
     sh = PREPARE_SHAPE
     byt = n * sh["H"] * (sh["d"] * 2 + sh["r"] * 2)
     return byt / el / 1e9, n, el
-
-
-def torch_float32():
-    import torch
-    return torch.float32
 
 
 def run_prepare(args, rank, world, local_rank):

@@ -200,3 +200,10 @@ def test_paged_validation():
     assert s(nslots=-3) == -1
     assert s(pt=MISALIGNED) == -2
     assert s(wsb=16) == -4
+
+
+def test_prefill_workspace_matches_header_note():
+    """lsa.h states about 3.26 GiB of prefill workspace for nq 4096, T 128K, B 2048."""
+    d = L.make_dims(1, 32, 8, 128, 64, 131072)
+    gib = L.lsa_prefill_workspace_size(d, 4096, 2048) / 2 ** 30
+    assert abs(gib - 3.26) < 0.01, gib
