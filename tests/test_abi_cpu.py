@@ -207,3 +207,17 @@ def test_prefill_workspace_matches_header_note():
     d = L.make_dims(1, 32, 8, 128, 64, 131072)
     gib = L.lsa_prefill_workspace_size(d, 4096, 2048) / 2 ** 30
     assert abs(gib - 3.26) < 0.01, gib
+
+
+def test_binding_argument_counts_match_header():
+    """Every ctypes signature has as many arguments as the lsa.h prototype."""
+    import re
+
+    text = open(L.HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    protos = re.findall(r"LSA_API\s+[\w\s\*]+?\b(lsa_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.S)
+    assert len(protos) == len(L._SIGS)
+    for name, params in protos:
+        params = params.strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert n == len(L._SIGS[name][1]), (name, n, len(L._SIGS[name][1]))
