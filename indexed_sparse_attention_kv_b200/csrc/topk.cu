@@ -543,13 +543,15 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster_kernel(const Top
     cluster.sync();   // keep this CTA's shared memory alive for remote readers
 }
 
-// Rows of at most NT * kSmallItems keys: one CTA per row holds the whole row
-// in registers and runs the exact block selection (radix passes on the order
-// keys, boundary ties to the lower position, ascending output through a
-// bitmap). Positions of coarse-to-fine candidates map through blkmap.
+// Rows of at most NT * ITEMS keys: one CTA per row holds the whole row in
+// registers (ITEMS per thread) and runs the exact block selection (radix
+// passes on the order keys, boundary ties to the lower position, ascending
+// output through a bitmap). Positions of coarse-to-fine candidates map
+// through blkmap. ITEMS is the smallest of 4 and 16 that holds the row, so
+// short rows do not loop over empty registers in every pass.
 constexpr int kSmallItems = 16;
 
-template <int NT>
+template <int NT, int ITEMS>
 __global__ void __launch_bounds__(NT) topk_small_kernel(const TopkArgs a) {
     __shared__ BlockSelShared sh;
     extern __shared__ uint32_t sbitmap[];
@@ -557,9 +559,9 @@ __global__ void __launch_bounds__(NT) topk_small_kernel(const TopkArgs a) {
     const float* src = a.scores + (size_t)row * a.n;
     pdl_launch_dependents();
     pdl_wait();   // the scores come from the previous kernel
-    uint32_t kk[kSmallItems];
+    uint32_t kk[ITEMS];
 #pragma unroll
-    for (int it = 0; it < kSmallItems; ++it) {
+    for (int it = 0; it < ITEMS; ++it) {
         const int i = (int)threadIdx.x + it * NT;
         kk[it] = i < a.n ? score_key(__ldcg(src + i)) : 0u;
     }
@@ -569,17 +571,17 @@ __global__ void __launch_bounds__(NT) topk_small_kernel(const TopkArgs a) {
     select_and_emit<NT>(
         [&](auto f) {
 #pragma unroll
-            for (int it = 0; it < kSmallItems; ++it)
+            for (int it = 0; it < ITEMS; ++it)
                 if (kk[it]) f(kk[it], (uint32_t)((int)threadIdx.x + it * NT));
         },
         a.B, a.n, sh, sbitmap, a.idx + (size_t)row * a.B,
         a.B, [&](int i) -> int32_t { return bm ? bm[i / a.blk] * a.blk + i % a.blk : i; });
 }
 
-template <int NT>
+template <int NT, int ITEMS>
 cudaError_t launch_small(const LaunchCtx& ctx, const TopkArgs& a, int rows) {
     const int smem = (a.n + 31) / 32 * 4;
-    auto kern = topk_small_kernel<NT>;
+    auto kern = topk_small_kernel<NT, ITEMS>;
     cudaError_t e = ensure_dyn_smem((const void*)kern, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
@@ -613,7 +615,8 @@ cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int
     // rows of up to 16K keys: one 1024-thread CTA per row (measured faster
     // than 256 or 512 threads for 4K-key rows: the selection's passes and
     // barriers, not the loads, set its time)
-    if (n <= 1024 * kSmallItems) return launch_small<1024>(ctx, a, rows);
+    if (n <= 1024 * 4) return launch_small<1024, 4>(ctx, a, rows);
+    if (n <= 1024 * kSmallItems) return launch_small<1024, kSmallItems>(ctx, a, rows);
     // Cluster size: about 16K keys per CTA, at most 8 (portable); fewer CTAs
     // per row when there are many rows.
     int cs = 1;
