@@ -155,7 +155,10 @@ LSA_API lsa_status lsa_indexed_attn(const lsa_dims* dims, const lsa_bf16* q, con
  *     one-time setup: it looks up the buffer's device address, zero-fills the
  *     buffer on `stream` and waits for `stream`. Make that first call before
  *     any stream capture begins; a first call on a capturing stream returns
- *     LSA_ERR_CUDA and enqueues nothing.
+ *     LSA_ERR_CUDA and enqueues nothing. The setup is kept for the life of
+ *     the process and is not redone after cudaDeviceReset (which reloads the
+ *     library's device image elsewhere): do not call this entry point on a
+ *     device after resetting it.
  *   - Only the merge counters at the start of the buffer must be zero when a
  *     call starts; the setup zeroes them and every completed call leaves
  *     them at zero. The partials need no initial value.

@@ -19,7 +19,7 @@ Sources (page title, then the passage):
   * Latent Sparse Attention: Towards Subquadratic Ultra-Long Context
     Attention, summary: queries score clusters instead of every key.
 
-Readings where the pages are silent (each is also listed in the design notes):
+Readings where the pages are silent:
   * query head i belongs to KV head i // G (contiguous GQA groups);
   * the B-th largest score is the threshold; every position above it is kept,
     and ties at the threshold go to the lower position (lower block index in

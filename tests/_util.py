@@ -9,8 +9,12 @@ import torch
 import oracle.lsa_oracle as O
 from indexed_sparse_attention_kv_b200 import inputs as I
 
-# Attention outputs: |gpu - oracle| <= ATOL elementwise, and the largest error
-# relative to the largest reference magnitude <= RTOL. Index sets: bit-exact.
+# Attention outputs ("within 1e-2 max-abs and 1e-2 relative of the oracle"),
+# checked three ways: every element |gpu - ref| <= ATOL + RTOL * |ref|; the
+# largest error <= ATOL; and the largest error relative to the largest
+# reference magnitude <= RTOL (binding when outputs are small). A purely
+# per-element relative bound is not used: an output element near zero has no
+# meaningful relative error after the bf16 store. Index sets: bit-exact.
 ATOL = 1e-2
 RTOL = 1e-2
 
@@ -26,6 +30,9 @@ def assert_out_close(gpu: torch.Tensor, ref: np.ndarray, what: str = "out") -> N
     mx = float(err.max()) if err.size else 0.0
     scale = float(np.abs(ref).max()) if ref.size else 0.0
     assert np.isfinite(g).all(), f"{what}: non-finite GPU output"
+    bad = err > ATOL + RTOL * np.abs(ref)
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements outside atol + rtol*|ref|, first at " \
+        f"{np.argwhere(bad)[0].tolist()}"
     assert mx <= ATOL, f"{what}: max abs err {mx:.3e} > {ATOL}"
     if scale > 0:
         assert mx / scale <= RTOL, f"{what}: max rel err {mx / scale:.3e} > {RTOL}"

@@ -279,6 +279,8 @@ def check_golden(o):
     assert np.array_equal(o.project_rows(x, P, g["G"]), np.array(g["exact"], dtype=np.float64))
     assert np.array_equal(o.round_to_bf16(o.project_rows(x, P, g["G"])), np.array(g["bf16"], dtype=np.float64))
     assert np.array_equal(o.round_to_e4m3(o.project_rows(x, P, g["G"])), np.array(g["e4m3"], dtype=np.float64))
+    assert np.array_equal(o.project_bf16(x, P, g["G"]), np.array(g["bf16"], dtype=np.float64))
+    assert np.array_equal(o.project_e4m3(x, P, g["G"]), np.array(g["e4m3"], dtype=np.float64))
     c = o.update_centroids(np.array(g["centroid_start"], dtype=np.float64), np.array(g["kt"], dtype=np.float64),
                            g["t0"], g["n"], g["blk"])
     assert np.array_equal(c, np.array(g["centroid_end"], dtype=np.float64))
@@ -416,6 +418,112 @@ def check_update_centroids(o):
     assert c3[0, 0, 0] == 256.0, c3
 
 
+def check_prefill_attention_rows(o):
+    """Every prefill row attends over its own index sets: row n equals torch
+    SDPA (fp64) on the K/V rows gathered by idx[n], with a different set for
+    every row and some rows padded with -1."""
+    rng = np.random.default_rng(28)
+    n, T, hkv, hq, d, B = 6, 30, 2, 8, 8, 7
+    G = hq // hkv
+    q = rng.standard_normal((n, hq, d))
+    k = rng.standard_normal((T, hkv, d)) * 2
+    v = rng.standard_normal((T, hkv, d))
+    idx = np.full((n, hkv, B), -1)
+    for i in range(n):
+        for h in range(hkv):
+            m = B - (i % 3)
+            idx[i, h, :m] = np.sort(rng.choice(T, m, replace=False))
+    assert len({idx[i].tobytes() for i in range(n)}) == n
+    got = o.prefill_attention(q, k, v, idx, 0.3)
+    assert got.shape == (n, hq, d)
+    for i in range(n):
+        for h in range(hkv):
+            sel = torch.as_tensor(idx[i, h][idx[i, h] >= 0])
+            kh = torch.as_tensor(k[:, h, :]).index_select(0, sel)
+            vh = torch.as_tensor(v[:, h, :]).index_select(0, sel)
+            qh = torch.as_tensor(q[i, h * G:(h + 1) * G])
+            want = _sdpa(qh[:, None, :], kh[None], vh[None], 0.3)[:, 0, :].numpy()
+            assert np.allclose(got[i, h * G:(h + 1) * G], want, rtol=1e-12, atol=1e-12), (i, h)
+
+
+def _int_dot_bruteforce(x, P, G):
+    """Projections from integer numerators with Python ints: x = X / 16 and
+    P = Q / 4 give y = (X . Q) / 64 exactly."""
+    X = np.rint(np.asarray(x) * 16).astype(np.int64)
+    Q = np.rint(np.asarray(P) * 4).astype(np.int64)
+    y = np.zeros(X.shape[:-1] + (Q.shape[1],))
+    for idx in np.ndindex(*X.shape[:-1]):
+        i = idx[-1]
+        for j in range(Q.shape[1]):
+            y[idx + (j,)] = sum(int(a) * int(b) for a, b in zip(X[idx], Q[i // G, j])) / 64
+    return y
+
+
+def check_project_casts(o):
+    """The cached projection rows are the exact dot products rounded once:
+    on inputs whose exact projections are fp32 values (multiples of 1/64
+    below 2^10), torch's fp32 -> float8_e4m3fn and -> bfloat16 casts are the
+    reference for project_e4m3 and project_bf16 (JSSA, Fig. 10: the
+    projected-key cache held in FP8); plus hand-derived E4M3 ties (17 -> 16,
+    19 -> 20) and saturation (+-1000 -> +-448) through a unit basis."""
+    rng = np.random.default_rng(29)
+    nb, G, d, r = 2, 2, 16, 8
+    x = rng.integers(-40, 41, size=(5, nb * G, d)) / 16.0
+    P = rng.integers(-3, 4, size=(nb, r, d)) / 4.0
+    exact = _int_dot_bruteforce(x, P, G)
+    assert np.abs(exact).max() < 448
+    e32 = torch.from_numpy(exact.astype(np.float32))
+    assert np.array_equal(e32.double().numpy(), exact)                # exact in fp32
+    want8 = e32.to(torch.float8_e4m3fn).double().numpy()
+    want16 = e32.to(torch.bfloat16).double().numpy()
+    assert (want8 != exact).sum() > 20 and (want16 != exact).sum() > 5   # rounding is exercised
+    assert np.array_equal(o.project_e4m3(x, P, G), want8)
+    assert np.array_equal(o.project_bf16(x, P, G), want16)
+    unit = np.zeros((1, 2, 4))
+    unit[0, 0, 0] = unit[0, 1, 3] = 1.0
+    xs = np.array([[[17.0, 0, 0, 19.0]], [[1000.0, 0, 0, -1000.0]], [[-17.0, 5, 5, 0.4375]]])
+    got = o.project_e4m3(xs, unit, 1)
+    assert np.array_equal(got[:, 0, :], [[16.0, 20.0], [448.0, -448.0], [-16.0, 0.4375]]), got
+
+
+def check_decode_step_bruteforce(o):
+    """A whole decode step against brute force: integer group scores with
+    Python ints, selection by lexicographic sort (score desc, position asc),
+    the set ascending, and SDPA (fp64) over the gathered rows; in the
+    coarse-to-fine mode, blocks by (block score desc, block index asc) first."""
+    rng = np.random.default_rng(30)
+    cases = [(8, 2, 60, 4, 16, 9, 0, 0), (4, 1, 33, 3, 8, 33, 0, 0), (6, 3, 20, 2, 8, 40, 0, 0),
+             (8, 2, 64, 3, 8, 10, 8, 3), (4, 1, 45, 2, 8, 12, 8, 2)]
+    for hq, hkv, T, r, d, B, blk, keep in cases:
+        G = hq // hkv
+        qt = rng.integers(-2, 3, size=(hq, r)).astype(np.float64)
+        kt = rng.integers(-2, 3, size=(T, hkv, r)).astype(np.float64)
+        q = rng.standard_normal((hq, d))
+        k = rng.standard_normal((T, hkv, d))
+        v = rng.standard_normal((T, hkv, d))
+        scale = 1.0 / math.sqrt(d)
+        idx, out = o.decode_step(q, qt, k, v, kt, B, scale, blk=blk, keep=keep)
+        assert idx.shape == (hkv, B) and out.shape == (hq, d)
+        for h in range(hkv):
+            s = np.array([sum(int(qt[i, j]) * int(kt[t, h, j]) for i in range(h * G, (h + 1) * G)
+                              for j in range(r)) for t in range(T)])
+            cand = np.arange(T)
+            if blk:
+                nblk = -(-T // blk)
+                bs = np.array([s[j * blk:(j + 1) * blk].sum() for j in range(nblk)])
+                blocks = np.lexsort((np.arange(nblk), -bs))[:keep]
+                cand = np.concatenate([np.arange(j * blk, min(T, (j + 1) * blk)) for j in blocks])
+            order = np.lexsort((cand, -s[cand]))[:B]
+            want = np.full(B, -1)
+            want[:len(order)] = np.sort(cand[order])
+            assert np.array_equal(idx[h], want), (hq, hkv, T, blk, h)
+            sel = torch.as_tensor(want[want >= 0])
+            kh = torch.as_tensor(k[:, h, :]).index_select(0, sel)
+            vh = torch.as_tensor(v[:, h, :]).index_select(0, sel)
+            ref = _sdpa(torch.as_tensor(q[h * G:(h + 1) * G])[:, None, :], kh[None], vh[None], scale)
+            assert np.allclose(out[h * G:(h + 1) * G], ref[:, 0, :].numpy(), rtol=1e-12, atol=1e-12)
+
+
 CHECKS = [
     check_select_bruteforce, check_select_special, check_scores_bruteforce, check_scores_onehot,
     check_attention_full_budget_sdpa, check_attention_subset_sdpa, check_attention_closed_forms,
@@ -423,6 +531,7 @@ CHECKS = [
     check_prefill_vs_decode_prefix, check_golden,
     check_round_bf16, check_round_e4m3, check_project_shifted_unit_basis, check_project_orthonormal,
     check_project_integer_exact, check_update_centroids, check_paged_attention,
+    check_prefill_attention_rows, check_project_casts, check_decode_step_bruteforce,
 ]
 
 
@@ -623,7 +732,53 @@ def _paged_inverse(q, k_pool, v_pool, slots, idx, scale):   # reads the table ba
     return O.indexed_attention(q, O.paged_rows(k_pool, inv), O.paged_rows(v_pool, inv), idx, scale)
 
 
+def _prefill_attn_row0(q_rows, k, v, idx, scale):   # every row uses row 0's index sets
+    return O.prefill_attention(q_rows, k, v, np.broadcast_to(np.asarray(idx)[:1], np.shape(idx)), scale)
+
+
+def _prefill_attn_shifted(q_rows, k, v, idx, scale):   # row n uses row n-1's index sets
+    idx = np.asarray(idx)
+    return O.prefill_attention(q_rows, k, v, np.concatenate([idx[:1], idx[:-1]]), scale)
+
+
+def _e4m3_proj_as_bf16(x, P, G):           # the FP8 cache rounded to bf16 instead
+    return O.round_to_bf16(O.project_rows(x, P, G))
+
+
+def _e4m3_proj_truncates(x, P, G):         # E4M3 rounding toward zero
+    y = O.project_rows(x, P, G)
+    m, e = np.frexp(np.abs(y))
+    ulp = np.ldexp(1.0, np.maximum(e - 1, -6) - 3)
+    return np.clip(np.sign(y) * np.floor(np.abs(y) / ulp) * ulp, -448, 448)
+
+
+def _step_unsorted(q, qt, k, v, kt, B, scale, blk=0, keep=0):   # the set left in score order
+    idx, out = O.decode_step(q, qt, k, v, kt, B, scale, blk=blk, keep=keep)
+    s = O.candidate_scores(O.group_mean_query(qt, kt.shape[1]), kt)
+    idx = idx.copy()
+    for h in range(idx.shape[0]):
+        sel = idx[h][idx[h] >= 0]
+        idx[h, :len(sel)] = sel[np.argsort(-s[h, sel], kind="stable")]
+    return idx, out
+
+
+def _step_ignores_hierarchy(q, qt, k, v, kt, B, scale, blk=0, keep=0):   # always flat
+    return O.decode_step(q, qt, k, v, kt, B, scale)
+
+
+def _step_other_group_query(q, qt, k, v, kt, B, scale, blk=0, keep=0):   # attention with head i's query shifted by one
+    idx, _ = O.decode_step(q, qt, k, v, kt, B, scale, blk=blk, keep=keep)
+    return idx, O.indexed_attention(np.roll(np.asarray(q), 1, axis=0), k, v, idx, scale)
+
+
 MUTANTS = {
+    "prefill_rows_use_row0_idx": dict(prefill_attention=_prefill_attn_row0),
+    "prefill_rows_shifted_idx": dict(prefill_attention=_prefill_attn_shifted),
+    "project_e4m3_rounds_to_bf16": dict(project_e4m3=_e4m3_proj_as_bf16),
+    "project_e4m3_truncates": dict(project_e4m3=_e4m3_proj_truncates),
+    "decode_step_set_unsorted": dict(decode_step=_step_unsorted),
+    "decode_step_ignores_hierarchy": dict(decode_step=_step_ignores_hierarchy),
+    "decode_step_rolled_queries": dict(decode_step=_step_other_group_query),
     "paged_table_inverted": dict(indexed_attention_paged=_paged_inverse),
     "bf16_truncates": dict(round_to_bf16=_bf16_truncate),
     "bf16_ties_away": dict(round_to_bf16=_bf16_ties_away),
