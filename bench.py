@@ -15,9 +15,9 @@ Multi-GPU: the decode step shards by sequence and KV head with no exchange, so
 each rank runs its own full workload (weak scaling, no data-path collective);
 `value` is the steps of all ranks divided by the slowest rank's time.
 
---impl reference times the CPU oracle (fp64 NumPy) on this host's cores on a
-bounded sample of the same workload (one (sequence, KV head) unit per step),
-scaled to whole decode steps.
+--impl reference times the CPU oracle (fp64 NumPy) on this host's cores: whole
+oracle decode steps for the decode lines (about 1.4 s each at 128K), bounded
+samples scaled to whole steps for the prefill and the projection.
 """
 from __future__ import annotations
 
@@ -261,87 +261,101 @@ def cpu_oracle_sample(w, x, budget_s=12.0, max_units=None):
     return done / units_per_step / elapsed, done, elapsed
 
 
+def parallelism(world):
+    return f"replicas{world}" if world > 1 else "single"
+
+
+def decode_config(w, world, fp8=False, paged=False):
+    """The `config` of a decode_128k line (either arm)."""
+    return config_dict(w, {"parallelism": parallelism(world),
+                           **({"workload": "decode_128k_fp8", "kt_dtype": "fp8_e4m3"} if fp8 else {}),
+                           **({"workload": "decode_128k_paged",
+                               "kv_layout": "pools [batch*T, hkv, d] bf16, page size 1, page table "
+                                            "[batch, T] int32 (a random permutation of the slots)"}
+                              if paged else {})})
+
+
+def resident_config(w, world):
+    return {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "d": w.d, "T": w.T,
+            "r": w.r, "B": w.B, "blk": w.blk, "keep": w.keep,
+            "l2": "256 MiB L2 flush after every step, timed alone and subtracted",
+            "parallelism": parallelism(world)}
+
+
+def prefill_config(w, world):
+    return {"workload": w.name, "nq": w.nq, "q_start": w.T - w.nq, "T": w.T, "hq": w.hq, "hkv": w.hkv,
+            "d": w.d, "r": w.r, "B": w.B, "l2": "inputs exceed L2 (128 MiB projected keys, 512 MiB K/V)",
+            "parallelism": parallelism(world)}
+
+
+def prepare_config(world):
+    return {"workload": "prepare_128k", **PREPARE_SHAPE, "nbases": PREPARE_SHAPE["H"],
+            "l2": "inputs exceed L2 (1 GiB of keys per step)", "parallelism": parallelism(world)}
+
+
 def run_reference(args, rank, world):
-    """Reference arm: the CPU oracle as it stands, on this host's cores."""
+    """Reference arm: the CPU oracle as it stands, on this host's cores.
+
+    Each timed step is one whole oracle decode step (all (sequence, KV head)
+    units) for the decode lines, which take about a second; for the prefill
+    and the projection, whose whole step takes hours on the host, each timed
+    step is a bounded sample of the workload and `value` is scaled from it.
+    Either way `ms_per_step` is the measured time of one timed step, so
+    steps x ms_per_step is the timed region."""
     if rank != 0:
         return 0
     from indexed_sparse_attention_kv_b200 import inputs as I
 
+    cores = blas_threads()
+    K, W = max(1, args.steps), max(1, args.warmup)
+
+    def line(metric, value, unit, ms_step, config, sample):
+        return {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
+                "steps": K, "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+                "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
     if args.workload in RESIDENT_METRICS:
         w = I.workload(args.workload)
         x = I.make_decode_inputs(w)
-        cpu_unit_sample(w, x, budget_s=0.0, max_units=max(1, args.warmup))
-        v, n, el = cpu_unit_sample(w, x, budget_s=0.0, max_units=max(1, args.steps))
-        line = {
-            "impl": "reference", "metric": RESIDENT_METRICS[w.name], "value": v, "unit": UNIT,
-            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "d": w.d, "T": w.T,
-                       "r": w.r, "B": w.B, "blk": w.blk, "keep": w.keep},
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"{n} (sequence, KV head) units per timed run, scaled to whole steps"},
-            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        }
-        print(json.dumps(line), flush=True)
-        return 0
-    if args.workload == "prepare_128k":
+        units = w.batch * w.hkv
+        for _ in range(W):
+            cpu_unit_sample(w, x, budget_s=math.inf, max_units=units)
+        el = sum(cpu_unit_sample(w, x, budget_s=math.inf, max_units=units)[2] for _ in range(K))
+        out = line(RESIDENT_METRICS[w.name], K / el, UNIT, el / K * 1e3, resident_config(w, world),
+                   f"{K} whole decode steps ({units} (sequence, KV head) units each)")
+    elif args.workload == "prepare_128k":
         sh = PREPARE_SHAPE
         hx = I.make_projection_inputs(PREPARE_SEED, 1, 4096, sh["H"], sh["d"], sh["r"], sh["H"], None, None)
-        cpu_prepare_sample(hx["x"], hx["P"], budget_s=0.0, max_tokens=256 * max(1, args.warmup))
-        v, n, el = cpu_prepare_sample(hx["x"], hx["P"], budget_s=0.0, max_tokens=256 * max(1, args.steps))
-        byt = prepare_bytes(sh)
-        line = {
-            "impl": "reference", "metric": PREPARE_METRIC, "value": v, "unit": PREPARE_UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": byt / (v * 1e9) * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "prepare_128k", **sh, "nbases": sh["H"]},
-            "cpu_baseline": {"value": v, "unit": PREPARE_UNIT, "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"{n} token rows x 8 KV heads per timed run, same algorithmic bytes per row"},
-            "e2e": {"value": v, "unit": PREPARE_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        }
-        print(json.dumps(line), flush=True)
-        return 0
-    if args.workload == "prefill_128k":
+        per = 4096
+        cpu_prepare_sample(hx["x"], hx["P"], budget_s=math.inf, max_tokens=per * W)
+        v, n, el = cpu_prepare_sample(hx["x"], hx["P"], budget_s=math.inf, max_tokens=per * K)
+        out = line(PREPARE_METRIC, v, PREPARE_UNIT, el / K * 1e3, prepare_config(world),
+                   f"each timed step projects {per} token rows x {sh['H']} KV heads ({n} rows in all); "
+                   f"GB/s of the same algorithmic bytes per row")
+    elif args.workload == "prefill_128k":
         w = I.workload("prefill_128k")
         x = I.make_prefill_inputs(w)
-        cpu_prefill_sample(w, x, budget_s=0.0, max_rows=max(1, args.warmup))
-        v, n, el = cpu_prefill_sample(w, x, budget_s=0.0, max_rows=max(1, args.steps))
-        line = {
-            "impl": "reference", "metric": PREFILL_METRIC, "value": v, "unit": PREFILL_UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "nq": w.nq, "T": w.T, "hq": w.hq, "hkv": w.hkv, "d": w.d, "r": w.r,
-                       "B": w.B},
-            "cpu_baseline": {"value": v, "unit": PREFILL_UNIT, "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"{n} query rows of 4096 per timed run, scaled to whole prefills"},
-            "e2e": {"value": v, "unit": PREFILL_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        }
-        print(json.dumps(line), flush=True)
-        return 0
-    w = I.workload(WORKLOAD)
-    x = I.make_decode_inputs(w)
-    cores = blas_threads()
-    # warm-up: W units; timed: K steps, each one (sequence, KV head) unit
-    cpu_oracle_sample(w, x, budget_s=0.0, max_units=max(1, args.warmup))
-    per_unit = []
-    for _ in range(args.steps):
-        v, n, el = cpu_oracle_sample(w, x, budget_s=0.0, max_units=1)
-        per_unit.append(el)
-    unit_s = sum(per_unit) / len(per_unit)
-    step_s = unit_s * w.batch * w.hkv
-    value = 1.0 / step_s
-    line = {
-        "impl": "reference",
-        "metric": {"decode_128k_fp8": METRIC_FP8, "decode_128k_paged": METRIC_PAGED}.get(args.workload, METRIC),
-        "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(w),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{args.steps} timed (sequence, KV head) units of 32 per step, scaled x32"},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line), flush=True)
+        per = 2
+        cpu_prefill_sample(w, x, budget_s=math.inf, max_rows=per * W)
+        v, n, el = cpu_prefill_sample(w, x, budget_s=math.inf, max_rows=per * K)
+        out = line(PREFILL_METRIC, v, PREFILL_UNIT, el / K * 1e3, prefill_config(w, world),
+                   f"each timed step runs {per} of the {w.nq} query rows (index + attention; {n} rows in all), "
+                   f"scaled to whole prefills")
+    else:
+        w = I.workload(WORKLOAD)
+        x = I.make_decode_inputs(w)
+        units = w.batch * w.hkv
+        for _ in range(W):
+            cpu_oracle_sample(w, x, budget_s=math.inf, max_units=units)
+        el = sum(cpu_oracle_sample(w, x, budget_s=math.inf, max_units=units)[2] for _ in range(K))
+        metric = {"decode_128k_fp8": METRIC_FP8, "decode_128k_paged": METRIC_PAGED}.get(args.workload, METRIC)
+        out = line(metric, K / el, UNIT, el / K * 1e3,
+                   decode_config(w, world, fp8=args.workload == "decode_128k_fp8",
+                                 paged=args.workload == "decode_128k_paged"),
+                   f"{K} whole decode steps ({units} (sequence, KV head) units each)")
+    print(json.dumps(out), flush=True)
     return 0
 
 
@@ -519,12 +533,7 @@ def run_ours(args, rank, world, local_rank):
             "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_dict(w, {"parallelism": f"replicas{world}" if world > 1 else "single",
-                                      **({"workload": "decode_128k_fp8", "kt_dtype": "fp8_e4m3"} if fp8 else {}),
-                                      **({"workload": "decode_128k_paged",
-                                          "kv_layout": "pools [batch*T, hkv, d] bf16, page size 1, page table "
-                                                       "[batch, T] int32 (a random permutation of the slots)"}
-                                         if paged else {})}),
+            "config": decode_config(w, world, fp8=fp8, paged=paged),
             "roofline": {"bound": "hbm", "kernel": "score_q64_kernel (lsa_score_fp8)" if fp8 else
                          "score_q64_kernel (lsa_score)", "achieved": achieved, "peak": peak,
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
@@ -704,10 +713,7 @@ def run_resident(args, rank, world, local_rank):
             "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "d": w.d, "T": w.T,
-                       "r": w.r, "B": w.B, "blk": w.blk, "keep": w.keep,
-                       "l2": "256 MiB L2 flush after every step, timed alone and subtracted",
-                       "parallelism": f"replicas{world}" if world > 1 else "single"},
+            "config": resident_config(w, world),
             "roofline": {"bound": "hbm", "kernel": "lsa_decode_step (whole step)", "achieved": achieved,
                          "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
                          "peak_kind": peak_kind, "algorithmic_bytes_per_launch": step_bytes,
@@ -865,9 +871,7 @@ def run_prefill(args, rank, world, local_rank):
             "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
             "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "nq": w.nq, "q_start": q0, "T": w.T, "hq": w.hq, "hkv": w.hkv,
-                       "d": w.d, "r": w.r, "B": w.B,
-                       "l2": "inputs exceed L2 (128 MiB projected keys, 512 MiB K/V)"},
+            "config": prefill_config(w, world),
             "roofline": {"bound": "tensor", "kernel": "lsa_prefill_index (score GEMMs + selection)",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "traffic": None, "peak_kind": peak_kind, "algorithmic_flop_per_launch": flop,
@@ -1025,8 +1029,7 @@ def run_prepare(args, rank, world, local_rank):
             "metric": PREPARE_METRIC, "value": achieved * world, "unit": PREPARE_UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": per_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "prepare_128k", **sh, "nbases": sh["H"],
-                       "l2": "inputs exceed L2 (1 GiB of keys per step)"},
+            "config": prepare_config(world),
             "roofline": {"bound": "hbm", "kernel": "project_kernel (lsa_project)", "achieved": achieved,
                          "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": project_traffic(),
                          "peak_kind": peak_kind, "algorithmic_bytes_per_launch": byt, "avg_launch_ms": per_ms},
@@ -1061,6 +1064,27 @@ def run_ncu_case(args):
             lsa.lsa_project(xd, Pd, y=y)
         torch.cuda.synchronize()
         print(f"ncu case project: {args.warmup}+{args.steps} launches")
+        return 0
+    if args.ncu_case in ("prefill_mid", "prefill_attn_mid"):
+        # mid-size prefill: T = 65536 keys, 1024 causal queries at T-1024..T-1, 32 / 8 heads, r 64,
+        # B 2048, integer-valued bf16 scoring inputs (80 MiB of K/V, 8 MiB of projected keys)
+        w = I.Workload("prefill_mid", 77, batch=1, hq=32, hkv=8, d=128, T=65536, r=64, B=2048, nq=1024)
+        x = I.make_prefill_inputs(w)
+        qt, kt = x["qt"].cuda(), x["kt"].cuda()
+        q0 = int(x["q_start"])
+        dims = _lib.prefill_dims(w.hq, kt)
+        ws = lsa.prefill_workspace(dims, w.nq, w.B)
+        idx = lsa.lsa_prefill_index(qt, kt, q0, w.B, ws=ws)
+        if args.ncu_case == "prefill_attn_mid":
+            q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+            out = torch.empty_like(q)
+            fn = lambda: lsa.lsa_prefill_attn(q, k, v, idx, out=out, ws=ws)  # noqa: E731
+        else:
+            fn = lambda: lsa.lsa_prefill_index(qt, kt, q0, w.B, idx=idx, ws=ws)  # noqa: E731
+        for _ in range(args.warmup + args.steps):
+            fn()
+        torch.cuda.synchronize()
+        print(f"ncu case {args.ncu_case}: {args.warmup}+{args.steps} calls, status {lsa.lsa_read_device_status(ws)}")
         return 0
     w = I.workload(WORKLOAD).with_(batch=2, name="decode_128k_b2")
     x = I.make_decode_inputs(w)
@@ -1102,8 +1126,11 @@ def main(argv=None):
                          "(indexer + indexed attention), the L2-resident decode steps "
                          "llama8b_32k and hier_1m, or prepare_128k (scoring preparation: projecting the 128K "
                          "key cache, and the decode-time append)")
-    ap.add_argument("--ncu-case", choices=["score", "score8", "topk", "attn", "step", "project"], default=None,
-                    help="run one component on a reduced 128K case (batch 2) for an ncu capture; no JSON")
+    ap.add_argument("--ncu-case", choices=["score", "score8", "topk", "attn", "step", "project", "prefill_mid",
+                                           "prefill_attn_mid"], default=None,
+                    help="run one component on a reduced case for an ncu capture (batch 2 of the 128K decode; "
+                         "one 128K sequence for project; a 64K-key, 1024-query prefill for prefill_mid and "
+                         "prefill_attn_mid); no JSON")
     args = ap.parse_args(argv)
     if args.ncu_case:
         return run_ncu_case(args)

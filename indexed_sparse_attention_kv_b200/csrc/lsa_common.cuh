@@ -10,6 +10,11 @@ namespace lsa {
 constexpr int kStatusBadIndex = 1;   // mirrors LSA_DEV_BAD_INDEX
 constexpr int kStatusTimeout = 2;    // mirrors LSA_DEV_TIMEOUT
 
+// Bound of the waits that drain asynchronous copies or MMAs already issued
+// before a CTA gives up after a timeout: those always complete, so this bound
+// is only a last resort and does not follow the (debug-settable) wait limit.
+constexpr long long kDrainNs = 4000000000ll;   // 4 s
+
 // ---------------------------------------------------------------- bf16 bits
 // A 32-bit word holding two bf16 values: element 2k in the low half, 2k+1 in
 // the high half (little-endian). bf16 -> fp32 is exact: the bf16 bits are the

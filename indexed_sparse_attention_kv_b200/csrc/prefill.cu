@@ -173,6 +173,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         return __shfl_sync(0xffffffffu, ok, 0) != 0;
     };
 
+    // Issued asynchronous work, for the drain after an abort: TMA loads
+    // (producer lane) and the last accumulator / A-slot commits (MMA lane).
+    int a_issued = 0, b_issued = 0;
+    int last_acc = -1, last_as = -1;
+    uint32_t last_aph = 0, last_asph = 0;
     if (warp == 0) {   // ----------------------------------------------- TMA producer
         int it = 0, ui = 0;
         bool ok = true;
@@ -189,6 +194,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int at = 0; at < atoms; ++at)
                     tma_load_2d(Aslot + as * a_bytes + at * kBM * rb, &tmA, at * 64, un.h * a.nq_pad + un.rb * kBM,
                                 &afull[as]);
+                a_issued = ui + 1;
             }
             __syncwarp();
             for (int c = un.c0; c < un.c1; ++c) {
@@ -203,6 +209,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     mbar_arrive_expect_tx(&full[s], b_bytes);
                     for (int at = 0; at < atoms; ++at)
                         tma_load_2d(Bs + at * kBN * rb, &tmB, un.h * a.r + at * 64, c * kBN, &full[s]);
+                    b_issued = it + 1;
                 }
                 __syncwarp();
                 ++it;
@@ -212,8 +219,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!ok && lane == 0) fail();
     } else if (warp == 1) {   // ---------------------------------------- MMA issuer
         const int nk = a.r / 16;
-        int it = 0, ui = 0, last_acc = -1;
-        uint32_t last_aph = 0;
+        int it = 0, ui = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < a.nunits && ok; u += gridDim.x) {
             const Unit un = decode_unit(u, a);
@@ -254,13 +260,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!ok) break;
             if (lane == 0) tc_commit(&aempty[as]);   // A slot free once this unit's MMAs are done
             __syncwarp();
+            last_as = as;
+            last_asph = (uint32_t)(ui / a.a_slots) & 1u;
             ++ui;
         }
         if (!ok && lane == 0) fail();
-        // On an abort, let the last MMAs finish before TMEM is released.
-        if (lane == 0 && *abort_flag && last_acc >= 0)
-            mbar_wait_bounded(&tfull[last_acc], last_aph, a.wait_limit, nullptr);
-        __syncwarp();
     } else if (warp >= kEpiWarp0) {   // ------------------------------- epilogue
         const int ew = warp - kEpiWarp0;
         const int quarter = warp & 3;   // TMEM lanes this warp may access
@@ -377,6 +381,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!ok && lane == 0) fail();
     }
     __syncthreads();
+    if (*abort_flag) {
+        // Every role has stopped and any abort is visible. Before shared
+        // memory and TMEM are released, wait (with the fixed drain bound) for
+        // the work already issued: each barrier has at most one outstanding
+        // phase, its last issued one.
+        if (warp == 0 && lane == 0) {
+            for (int s = 0; s < a.stages && s < b_issued; ++s) {
+                const int last = s + ((b_issued - 1 - s) / a.stages) * a.stages;
+                mbar_wait_bounded(&full[s], (uint32_t)(last / a.stages) & 1u, kDrainNs);
+            }
+            for (int s = 0; s < a.a_slots && s < a_issued; ++s) {
+                const int last = s + ((a_issued - 1 - s) / a.a_slots) * a.a_slots;
+                mbar_wait_bounded(&afull[s], (uint32_t)(last / a.a_slots) & 1u, kDrainNs);
+            }
+        }
+        if (warp == 1 && lane == 0) {
+            // MMAs complete in order: the last accumulator commit covers them all
+            if (last_acc >= 0) mbar_wait_bounded(&tfull[last_acc], last_aph, kDrainNs);
+            if (last_as >= 0) mbar_wait_bounded(&aempty[last_as], last_asph, kDrainNs);
+        }
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tbase, kAccCols);

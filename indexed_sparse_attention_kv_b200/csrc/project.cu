@@ -131,6 +131,11 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         return __shfl_sync(0xffffffffu, ok, 0) != 0;
     };
 
+    // Issued asynchronous work, for the drain after an abort: TMA loads
+    // (producer lane) and the last accumulator / basis-slot commits (MMA lane).
+    long long x_issued = 0;
+    int p_issued = 0, last_acc = -1, last_ps = -1;
+    uint32_t last_aph = 0, last_psph = 0;
     if (warp == 0) {   // ----------------------------------------------- TMA producer
         int pi = -1, cur_basis = -1;
         bool ok = true;
@@ -149,6 +154,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                     for (int at = 0; at < a.atoms; ++at)
                         tma_load_2d(Pslot + ps * p_bytes + at * a.r * a.rb, &tmP, at * (a.rb / 2), t.basis * a.r,
                                     &pfull[ps]);
+                    p_issued = pi + 1;
                 }
                 __syncwarp();
             }
@@ -164,20 +170,24 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 for (int at = 0; at < a.atoms; ++at)
                     tma_load_2d(Xst + s * x_bytes + at * kPM * a.rb, &tmX, t.head * a.d + at * (a.rb / 2),
                                 (int)t.z0, &full[s]);
+                x_issued = it + 1;
             }
             __syncwarp();
         }
         if (!ok && lane == 0) fail();
     } else if (warp == 1) {   // ---------------------------------------- MMA issuer
         const uint32_t idesc = f16_idesc(kPM, a.r);
-        int pi = -1, cur_basis = -1, last_acc = -1;
-        uint32_t last_aph = 0;
+        int pi = -1, cur_basis = -1;
         bool ok = true;
         for (long long u = u0; u < u1 && ok; ++u) {
             const Tile t = decode_tile(u, a);
             if (t.basis != cur_basis) {
                 if (pi >= 0 && lane == 0) tc_commit(&pempty[pi & 1]);   // previous basis free after its MMAs
                 __syncwarp();
+                if (pi >= 0) {
+                    last_ps = pi & 1;
+                    last_psph = (uint32_t)(pi >> 1) & 1u;
+                }
                 ++pi;
                 cur_basis = t.basis;
                 if (!warp_wait(&pfull[pi & 1], (uint32_t)(pi >> 1) & 1u)) {
@@ -213,9 +223,6 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             last_aph = aph;
         }
         if (!ok && lane == 0) fail();
-        if (lane == 0 && *abort_flag && last_acc >= 0)
-            mbar_wait_bounded(&tfull[last_acc], last_aph, a.wait_limit, nullptr);
-        __syncwarp();
     } else if (warp >= kProjEpiWarp0) {   // ------------------------- epilogue
         const int quarter = warp & 3;     // TMEM lanes this warp may access
         const int row_in = quarter * 32 + lane;
@@ -270,6 +277,28 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         if (!ok && lane == 0) fail();
     }
     __syncthreads();
+    if (*abort_flag) {
+        // Every role has stopped and any abort is visible. Before shared
+        // memory and TMEM are released, wait (with the fixed drain bound) for
+        // the work already issued: each barrier has at most one outstanding
+        // phase, its last issued one.
+        if (warp == 0 && lane == 0) {
+            for (int s = 0; s < a.stages && s < x_issued; ++s) {
+                const long long last = s + ((x_issued - 1 - s) / a.stages) * a.stages;
+                mbar_wait_bounded(&full[s], (uint32_t)(last / a.stages) & 1u, kDrainNs);
+            }
+            for (int s = 0; s < 2 && s < p_issued; ++s) {
+                const int last = s + ((p_issued - 1 - s) / 2) * 2;
+                mbar_wait_bounded(&pfull[s], (uint32_t)(last >> 1) & 1u, kDrainNs);
+            }
+        }
+        if (warp == 1 && lane == 0) {
+            // MMAs complete in order: the last accumulator commit covers them all
+            if (last_acc >= 0) mbar_wait_bounded(&tfull[last_acc], last_aph, kDrainNs);
+            if (last_ps >= 0) mbar_wait_bounded(&pempty[last_ps], last_psph, kDrainNs);
+        }
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tbase, a.acc_cols);

@@ -22,7 +22,6 @@ constexpr int kScoreThreads = 256;
 constexpr int kScoreWarps = kScoreThreads / 32;
 constexpr int kScoreStages = 4;
 constexpr int kChunkTarget = 16384;   // bytes per pipeline stage (approximate)
-constexpr long long kDrainNs = 4000000000ll;   // 4 s: copies in flight always land
 
 struct ScoreArgs {
     const uint16_t* qt;    // [batch, hq, r]
@@ -330,10 +329,10 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_launch_dependents();   // the selection kernel may start its prologue
+    int issued = 0;            // bulk copies issued (producer lane)
     if (warp == kQConsumers) {
         if (lane == 0) {
             const uint64_t stream_pol = policy_evict_first();   // read-once stream: keep it out of L2's way
-            int issued = 0;
             for (int i = 0; i < nch; ++i) {
                 const int s = i % STAGES;
                 if (i >= STAGES &&
@@ -347,14 +346,6 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
                 mbar_arrive_expect_tx(&full[s], bytes);
                 bulk_g2s_hint(stages + s * kQChunk, kt_b + (size_t)t0 * token_bytes, bytes, &full[s], stream_pol);
                 issued = i + 1;
-            }
-            if (*abort_flag) {
-                // Leave no bulk copy in flight into this CTA's shared memory.
-                set_status(a.status, kStatusTimeout);
-                for (int s = 0; s < STAGES && s < issued; ++s) {
-                    const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
-                    mbar_wait_bounded(&full[s], (uint32_t)((last / STAGES) & 1), kDrainNs);
-                }
             }
         }
     } else {
@@ -428,6 +419,19 @@ __global__ void __launch_bounds__(kQThreads, 2) score_q64_kernel(const ScoreArgs
         }
     }
     __syncthreads();
+    if (*abort_flag) {
+        // Every role has stopped, and an abort from any of them is visible
+        // here. Leave no bulk copy in flight into this CTA's shared memory:
+        // each stage has at most one outstanding phase, its last issued one.
+        if (warp == kQConsumers && lane == 0) {
+            set_status(a.status, kStatusTimeout);
+            for (int s = 0; s < STAGES && s < issued; ++s) {
+                const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
+                mbar_wait_bounded(&full[s], (uint32_t)((last / STAGES) & 1), kDrainNs);
+            }
+        }
+        __syncthreads();
+    }
     if (HIST) {
         uint32_t* gh = a.ghist + (size_t)b * hkv * kHistBins;
         for (int e = threadIdx.x; e < hkv * kHistBins / 2; e += kQThreads) {
