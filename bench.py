@@ -44,6 +44,7 @@ UNIT = "steps/s"
 WORKLOAD = "decode_128k"
 FALLBACK_HBM_GBS = 6650.0
 KERNELS_PER_STEP = 3      # scorer, top-B, indexed attention (split combine fused into it)
+QUERY_SETS = 8            # decode steps cycle through this many query sets (8 x 32 MiB of rows > L2)
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 SCORER_SOURCES = ["indexed_sparse_attention_kv_b200/csrc/score.cu",
                   "indexed_sparse_attention_kv_b200/csrc/lsa_common.cuh"]
@@ -81,7 +82,8 @@ def _env_int(name, default):
 def config_dict(w, extra=None):
     d = {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "d": w.d, "T": w.T, "r": w.r,
          "B": w.B, "heavy_hitters": w.heavy_frac, "kv_layout": "[batch, T, hkv, d] bf16",
-         "l2": "inputs exceed L2 (each step streams the 512 MiB projected-key cache)"}
+         "l2": f"inputs exceed L2 (each step streams the 512 MiB projected-key cache; steps cycle through "
+               f"{QUERY_SETS} query sets, so each selects its own 32 MiB of K/V rows)"}
     if extra:
         d.update(extra)
     return d
@@ -390,22 +392,29 @@ def run_ours(args, rank, world, local_rank):
     idx = torch.empty((w.batch, w.hkv, w.B), dtype=torch.int32, device=dev)
     out = torch.empty_like(d["q"])
     stream = torch.cuda.current_stream(dev)
+    # Successive steps use different query sets: each step selects its own K/V
+    # rows, as consecutive decode steps of one layer do (with other layers in
+    # between), instead of re-reading the previous step's rows from L2.
+    qs = I.make_query_sets(w, QUERY_SETS, seed=rank_seed(w, rank) + 100)
+    dq, dqt = qs["q"].to(dev), qs["qt"].to(dev)
 
-    def step():
+    def step(i=None):
+        q = d["q"] if i is None else dq[i]
+        qt = d["qt"] if i is None else dqt[i]
         if fp8:
-            lsa.lsa_decode_step_fp8(d["q"], d["qt"], d["k"], d["v"], d["kt8"], w.B, idx_out=idx, out=out, ws=ws)
+            lsa.lsa_decode_step_fp8(q, qt, d["k"], d["v"], d["kt8"], w.B, idx_out=idx, out=out, ws=ws)
         elif paged:
-            lsa.lsa_decode_step_paged(d["q"], d["qt"], d["k_pool"], d["v_pool"], d["page_table"], d["kt"], w.B,
+            lsa.lsa_decode_step_paged(q, qt, d["k_pool"], d["v_pool"], d["page_table"], d["kt"], w.B,
                                       idx_out=idx, out=out, ws=ws)
         else:
-            lsa.lsa_decode_step(d["q"], d["qt"], d["k"], d["v"], d["kt"], w.B, idx_out=idx, out=out, ws=ws)
+            lsa.lsa_decode_step(q, qt, d["k"], d["v"], d["kt"], w.B, idx_out=idx, out=out, ws=ws)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    for _ in range(max(3, args.warmup)):
-        step()
+    for i in range(max(3, args.warmup)):
+        step(i % QUERY_SETS)
     torch.cuda.synchronize()
     status = lsa.lsa_read_device_status(ws)
 
@@ -418,10 +427,10 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         return g
 
-    # one decode step (3 kernel launches) captured once, replayed K times
-    g_step = graph_of(step)
-    for _ in range(max(3, args.warmup)):
-        g_step.replay()
+    # one decode step captured per query set, the graphs replayed in turn
+    g_steps = [graph_of(lambda i=i: step(i)) for i in range(QUERY_SETS)]
+    for i in range(max(3, args.warmup)):
+        g_steps[i % QUERY_SETS].replay()
     torch.cuda.synchronize()
 
     # ---- timed region: K whole decode steps
@@ -431,8 +440,8 @@ def run_ours(args, rank, world, local_rank):
         barrier()
         torch.cuda.synchronize()
         e0.record(stream)
-        for _ in range(args.steps):
-            g_step.replay()
+        for i in range(args.steps):
+            g_steps[i % QUERY_SETS].replay()
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -482,13 +491,13 @@ def run_ours(args, rank, world, local_rank):
     del graphs, flush
 
     # ---- end to end through the public API: H2D q, qt from pinned host, step, D2H out and idx
-    hq = x["q"].pin_memory()
-    hqt = x["qt"].pin_memory()
+    hq = qs["q"].pin_memory()
+    hqt = qs["qt"].pin_memory()
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     hidx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
-    for _ in range(2):
-        d["q"].copy_(hq, non_blocking=True)
-        d["qt"].copy_(hqt, non_blocking=True)
+    for i in range(2):
+        d["q"].copy_(hq[i], non_blocking=True)
+        d["qt"].copy_(hqt[i], non_blocking=True)
         step()
         hout.copy_(out, non_blocking=True)
         hidx.copy_(idx, non_blocking=True)
@@ -496,9 +505,9 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(args.steps):
-        d["q"].copy_(hq, non_blocking=True)
-        d["qt"].copy_(hqt, non_blocking=True)
+    for i in range(args.steps):
+        d["q"].copy_(hq[i % QUERY_SETS], non_blocking=True)
+        d["qt"].copy_(hqt[i % QUERY_SETS], non_blocking=True)
         step()
         hout.copy_(out, non_blocking=True)
         hidx.copy_(idx, non_blocking=True)
@@ -544,7 +553,7 @@ def run_ours(args, rank, world, local_rank):
             "components_ms": {"scoring": comp[0], "top_b": comp[1], "attention": comp[2]},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e, "unit": UNIT,
-                    "h2d_bytes_per_step": hq.numel() * 2 + hqt.numel() * 2,
+                    "h2d_bytes_per_step": (hq.numel() + hqt.numel()) * 2 // QUERY_SETS,
                     "d2h_bytes_per_step": hout.numel() * 2 + hidx.numel() * 4},
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "clocks": clocks,
@@ -640,8 +649,8 @@ def run_resident(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    for _ in range(max(3, args.warmup)):
-        step()
+    for i in range(max(3, args.warmup)):
+        step(i % QUERY_SETS)
     torch.cuda.synchronize()
     status = lsa.lsa_read_device_status(ws)
 
@@ -814,8 +823,8 @@ def run_prefill(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    for _ in range(max(3, args.warmup)):
-        step()
+    for i in range(max(3, args.warmup)):
+        step(i % QUERY_SETS)
     torch.cuda.synchronize()
     status = lsa.lsa_read_device_status(ws)
     e0 = torch.cuda.Event(enable_timing=True)

@@ -27,7 +27,7 @@ from dataclasses import dataclass, field, replace
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_decode_inputs", "make_prefill_inputs", "workload"]
+__all__ = ["Workload", "WORKLOADS", "make_decode_inputs", "make_prefill_inputs", "make_query_sets", "workload"]
 
 
 @dataclass(frozen=True)
@@ -143,6 +143,21 @@ def make_decode_inputs(w: Workload, seed: int | None = None) -> dict[str, torch.
                 k[b, p, h, :] = (k[b, p, h, :].float() * s).to(torch.bfloat16)
                 kt[b, p, h, :] = (kt[b, p, h, :].float() * s).to(torch.bfloat16)
     return {"q": q, "qt": qt, "k": k, "v": v, "kt": kt, "heavy": heavy}
+
+
+def make_query_sets(w: Workload, count: int, seed: int) -> dict[str, torch.Tensor]:
+    """`count` further decode queries for the same caches: q [count, batch, hq, d]
+    (N(0, 1) as bf16) and qt [count, batch, hq, r] (integers in [-R, R] as bf16),
+    set i drawn from seed + i in the order qt, q. Successive decode steps of a
+    benchmark use different sets, so that each step selects its own K/V rows
+    instead of re-reading the previous step's rows from L2."""
+    q = torch.empty((count, w.batch, w.hq, w.d), dtype=torch.bfloat16)
+    qt = torch.empty((count, w.batch, w.hq, w.r), dtype=torch.bfloat16)
+    for i in range(count):
+        gen = torch.Generator().manual_seed(seed + i)
+        qt[i] = _int_bf16((w.batch, w.hq, w.r), w.int_range, gen)
+        q[i] = _normal_bf16((w.batch, w.hq, w.d), gen)
+    return {"q": q, "qt": qt}
 
 
 def make_prefill_inputs(w: Workload, seed: int | None = None) -> dict[str, torch.Tensor]:
