@@ -308,6 +308,10 @@ def run_reference(args, rank, world):
         return 0
     from indexed_sparse_attention_kv_b200 import inputs as I
 
+    if args.workload in COMPARE_METRICS:
+        print(json.dumps({"impl": "reference", "unavailable": "comparison line: the oracle defines the method, not "
+                                                             "the comparison systems"}), flush=True)
+        return 0
     cores = blas_threads()
     K, W = max(1, args.steps), max(1, args.warmup)
 
@@ -570,6 +574,132 @@ def run_ours(args, rank, world, local_rank):
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "clocks": clocks,
             "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+COMPARE_METRICS = {
+    "full_kv_128k": "full-KV decode attention steps/s at 128K (comparison: dense attention over every cached "
+                    "position, the same attention kernel with index sets covering the whole cache)",
+    "gather_attend_128k": "gather-then-attend decode steps/s at 128K, B=2048 (comparison: the selected K/V rows "
+                          "copied to a dense buffer before attention)",
+}
+
+
+def run_compare(args, rank, world, local_rank):
+    """Comparison systems of the pages, measured with this library's kernels
+    (JSSA, Fig. 4: sparse decode against full-KV attention; Fig. 2b and Fig. 6:
+    gather-free attention against gather-then-attend). Each line also reports
+    the gather-free sparse path measured the same way in the same run."""
+    import torch
+    import torch.distributed as dist
+
+    import indexed_sparse_attention_kv_b200 as lsa
+    from indexed_sparse_attention_kv_b200 import _lib
+    from indexed_sparse_attention_kv_b200 import inputs as I
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    lsa.lib()
+    w = I.workload(WORKLOAD)
+    x = I.make_decode_inputs(w, seed=rank_seed(w, rank))
+    d = {k: x[k].to(dev) for k in ("q", "qt", "k", "v", "kt")}
+    qs = I.make_query_sets(w, QUERY_SETS, seed=rank_seed(w, rank) + 100)
+    dq, dqt = qs["q"].to(dev), qs["qt"].to(dev)
+    dims = _lib.decode_dims(d["q"], d["qt"], d["k"])
+    out = torch.empty_like(d["q"])
+    stream = torch.cuda.current_stream(dev)
+    full = args.workload == "full_kv_128k"
+    ws_step = lsa.workspace(dims, w.B, device=dev)
+    idx_out = torch.empty((w.batch, w.hkv, w.B), dtype=torch.int32, device=dev)
+
+    def sparse_step(i):   # the gather-free step (the product path)
+        lsa.lsa_decode_step(dq[i], dqt[i], d["k"], d["v"], d["kt"], w.B, idx_out=idx_out, out=out, ws=ws_step)
+
+    if full:
+        idx_all = torch.arange(w.T, dtype=torch.int32, device=dev).view(1, 1, w.T).expand(
+            w.batch, w.hkv, w.T).contiguous()
+        ws_full = lsa.workspace(dims, w.T, device=dev)
+
+        def cmp_step(i):
+            lsa.lsa_indexed_attn(dq[i], d["k"], d["v"], idx_all, out=out, ws=ws_full)
+
+        cmp_bytes = w.batch * w.T * w.hkv * w.d * 2 * 2 + w.batch * w.hq * w.d * 2 * 2
+    else:
+        scores = torch.empty((w.batch, w.hkv, w.T), dtype=torch.float32, device=dev)
+        idx = torch.empty((w.batch, w.hkv, w.B), dtype=torch.int32, device=dev)
+        kg = torch.empty((w.batch, w.B, w.hkv, w.d), dtype=torch.bfloat16, device=dev)
+        vg = torch.empty_like(kg)
+        bi = torch.arange(w.batch, device=dev).view(-1, 1, 1)
+        hi = torch.arange(w.hkv, device=dev).view(1, 1, -1)
+        idx_dense = torch.arange(w.B, dtype=torch.int32, device=dev).view(1, 1, w.B).expand(
+            w.batch, w.hkv, w.B).contiguous()
+        gdims = lsa.lsa_dims(w.batch, w.hq, w.hkv, w.d, w.r, w.B)
+        ws_g = lsa.workspace(gdims, w.B, device=dev)
+
+        def cmp_step(i):
+            lsa.lsa_score(dqt[i], d["kt"], scores)
+            lsa.lsa_topk(scores, w.B, idx)
+            it = idx.transpose(1, 2).long()           # [batch, B, hkv]
+            kg.copy_(d["k"][bi, it, hi])
+            vg.copy_(d["v"][bi, it, hi])
+            lsa.lsa_indexed_attn(dq[i], kg, vg, idx_dense, out=out, ws=ws_g)
+
+        cmp_bytes = algorithmic_bytes(w)[0] + 2 * algorithmic_bytes(w)[1] + algorithmic_bytes(w)[2]
+
+    def graph_of(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(QUERY_SETS):
+                fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        return g
+
+    for i in range(QUERY_SETS):
+        cmp_step(i)
+        sparse_step(i)
+    torch.cuda.synchronize()
+    g_cmp, g_sparse = graph_of(cmp_step), graph_of(sparse_step)
+    rounds = max(1, args.steps // QUERY_SETS)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    res = {}
+    with ClockSampler(dev) as clk:
+        for name, g in (("cmp", g_cmp), ("sparse", g_sparse)):
+            for _ in range(max(1, args.warmup // QUERY_SETS)):
+                g.replay()
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(rounds):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            res[name] = e0.elapsed_time(e1) / (rounds * QUERY_SETS)
+    clocks = clk.summary()
+    ms_cmp, ms_sparse = max_over_ranks([res["cmp"], res["sparse"]], world, dev)
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        steps = rounds * QUERY_SETS
+        line = {
+            "metric": COMPARE_METRICS[args.workload], "value": world * 1e3 / ms_cmp, "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": max(1, args.warmup // QUERY_SETS) * QUERY_SETS, "ms_per_step": ms_cmp,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**decode_config(w, world), "workload": args.workload},
+            "roofline": {"bound": "hbm", "kernel": "attn_kernel over every position" if full else
+                         "scorer + top-B + gather copy + attention", "achieved": cmp_bytes / (ms_cmp / 1e3) / 1e9,
+                         "peak": peak, "unit": "GB/s", "frac": cmp_bytes / (ms_cmp / 1e3) / 1e9 / peak,
+                         "traffic": None, "peak_kind": peak_kind, "algorithmic_bytes_per_launch": cmp_bytes,
+                         "avg_launch_ms": ms_cmp},
+            "gather_free_sparse_step_ms": ms_sparse,
+            "sparse_speedup": ms_cmp / ms_sparse,
+            "cpu_baseline": None,
+            "e2e": None,
+            "gpu_launches": (1 if full else 5) * steps,
+            "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     return 0
@@ -1140,13 +1270,15 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=["decode_128k", "decode_128k_fp8", "decode_128k_paged", "prefill_128k",
-                                           "llama8b_32k", "hier_1m", "prepare_128k"],
+                                           "llama8b_32k", "hier_1m", "prepare_128k", "full_kv_128k",
+                                           "gather_attend_128k"],
                     default="decode_128k",
                     help="decode_128k (the headline), decode_128k_fp8 (the same step over an FP8 projected-key "
                          "cache), decode_128k_paged (the same step with K/V in page-size-1 pools), prefill_128k "
                          "(indexer + indexed attention), the L2-resident decode steps "
-                         "llama8b_32k and hier_1m, or prepare_128k (scoring preparation: projecting the 128K "
-                         "key cache, and the decode-time append)")
+                         "llama8b_32k and hier_1m, prepare_128k (scoring preparation: projecting the 128K "
+                         "key cache, and the decode-time append), or the comparisons full_kv_128k (dense "
+                         "attention over the whole cache) and gather_attend_128k (selected rows copied first)")
     ap.add_argument("--ncu-case", choices=["score", "score8", "topk", "attn", "step", "project", "prefill_mid",
                                            "prefill_attn_mid"], default=None,
                     help="run one component on a reduced case for an ncu capture (batch 2 of the 128K decode; "
@@ -1176,6 +1308,8 @@ def main(argv=None):
             return run_prepare(args, rank, world, local_rank)
         if args.workload in RESIDENT_METRICS:
             return run_resident(args, rank, world, local_rank)
+        if args.workload in COMPARE_METRICS:
+            return run_compare(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:

@@ -30,7 +30,10 @@
  *     fewer than B candidates exist. NaN scores mark non-candidates.
  *   - Supported sizes: r in {16, 32, 64, 128}; d in {64, 128, 256};
  *     1 <= hkv, hkv * r <= 4096; G = hq / hkv in {1, 2, 4, 8, 16};
- *     1 <= T <= 2^31 - 1; 1 <= B <= 65536. Other sizes return
+ *     1 <= T <= 2^31 - 1; 1 <= B <= 65536 (the attention entries
+ *     lsa_indexed_attn, lsa_indexed_attn_paged and lsa_indexed_attn_noalloc,
+ *     which only read index sets, and lsa_workspace_size accept B <= 2^24, so
+ *     that one index set can cover a whole cache). Other sizes return
  *     LSA_ERR_UNSUPPORTED.
  *   - Errors found on the device (an index outside [-1, T), a bounded wait that
  *     ran out) are OR-ed into a status word at the start of the workspace;

@@ -62,6 +62,15 @@ lsa_status check_B(int B) {
     return LSA_OK;
 }
 
+// The attention entries only read index sets, so they accept longer ones (an
+// index set may cover a whole 128K cache: the dense full-KV comparison).
+constexpr int kMaxAttnB = 1 << 24;
+lsa_status check_B_attn(int B) {
+    if (B < 1) return LSA_ERR_ARG;
+    if (B > kMaxAttnB) return LSA_ERR_UNSUPPORTED;
+    return LSA_OK;
+}
+
 lsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA; }
 
 // Workspace layout (byte offsets from the 256-byte aligned base).
@@ -215,7 +224,7 @@ const char* lsa_status_string(lsa_status s) {
 void lsa_debug_set_wait_limit(long long ns) { g_wait_limit.store(ns < 0 ? kDefaultWaitLimit : ns); }
 
 size_t lsa_workspace_size(const lsa_dims* dims, int B, int blk, int nblk_keep) {
-    if (check_dims(dims) != LSA_OK || check_B(B) != LSA_OK) return 0;
+    if (check_dims(dims) != LSA_OK || check_B_attn(B) != LSA_OK) return 0;
     if (blk < 0 || nblk_keep < 0 || (blk > 0) != (nblk_keep > 0)) return 0;
     return decode_layout(dims, B, blk, nblk_keep, device_sms()).total;
 }
@@ -249,7 +258,7 @@ lsa_status lsa_indexed_attn(const lsa_dims* dims, const lsa_bf16* q, const lsa_b
                             void* stream) {
     lsa_status s = check_dims(dims);
     if (s != LSA_OK) return s;
-    if ((s = check_B(B)) != LSA_OK) return s;
+    if ((s = check_B_attn(B)) != LSA_OK) return s;
     if (!q || !k || !v || !idx || !out) return LSA_ERR_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(out)) return LSA_ERR_ALIGN;
     if (!std::isfinite(scale)) return LSA_ERR_ARG;
@@ -268,7 +277,7 @@ lsa_status lsa_indexed_attn_noalloc(const lsa_dims* dims, const lsa_bf16* q, con
                                     void* stream) {
     lsa_status s = check_dims(dims);
     if (s != LSA_OK) return s;
-    if ((s = check_B(B)) != LSA_OK) return s;
+    if ((s = check_B_attn(B)) != LSA_OK) return s;
     if (!q || !k || !v || !idx || !out) return LSA_ERR_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(out)) return LSA_ERR_ALIGN;
     if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0) return LSA_ERR_ALIGN;
@@ -358,7 +367,7 @@ lsa_status lsa_indexed_attn_paged(const lsa_dims* dims, const lsa_bf16* q, const
                                   int B, float scale, lsa_bf16* out, void* ws, size_t ws_bytes, void* stream) {
     lsa_status s = check_dims(dims);
     if (s != LSA_OK) return s;
-    if ((s = check_B(B)) != LSA_OK) return s;
+    if ((s = check_B_attn(B)) != LSA_OK) return s;
     if (!q || !k_pool || !v_pool || !page_table || !idx || !out || nslots < 1) return LSA_ERR_ARG;
     if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(page_table) || !aligned16(idx) ||
         !aligned16(out))

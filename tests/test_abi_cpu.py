@@ -71,6 +71,11 @@ def test_null_and_alignment():
                                 ALIGNED, 1 << 30, None) == -1
     assert lib.lsa_indexed_attn(ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, ALIGNED, 16, f(float("nan")),
                                 ALIGNED, ALIGNED, 1 << 30, None) == -1
+    # index sets longer than 65536 are read by the attention entries (up to 2^24), not selected
+    assert lib.lsa_indexed_attn(ctypes.byref(d), ALIGNED, ALIGNED, ALIGNED, ALIGNED, (1 << 24) + 1, f(0.1),
+                                ALIGNED, ALIGNED, 1 << 30, None) == -7
+    assert lib.lsa_workspace_size(ctypes.byref(d), 131072, 0, 0) > 0
+    assert lib.lsa_workspace_size(ctypes.byref(d), (1 << 24) + 1, 0, 0) == 0
     assert lib.lsa_block_centroids(ctypes.byref(d), ALIGNED, 0, ALIGNED, None) == -1
     assert lib.lsa_block_centroids(ctypes.byref(d), ALIGNED, 64, MISALIGNED, None) == -2
     assert lib.lsa_read_device_status(None, ALIGNED, None) == -1

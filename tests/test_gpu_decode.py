@@ -242,3 +242,16 @@ def test_named_workload_hier_1m():
     assert_out_close(out, ref_out)
     del dx, cen
     torch.cuda.empty_cache()
+
+
+def test_attention_over_a_whole_cache():
+    """An index set may cover every cached position (B = T > 65536): the
+    dense full-KV attention, equal to the oracle over all positions."""
+    w = I.Workload("whole_cache", 109, batch=1, hq=4, hkv=1, d=128, T=70000, r=64, B=70000)
+    x = I.make_decode_inputs(w)
+    dx = to_dev(x, ("q", "k", "v"))
+    idx = torch.arange(w.T, dtype=torch.int32, device="cuda").view(1, 1, w.T)
+    out = lsa.lsa_indexed_attn(dx["q"], dx["k"], dx["v"], idx)
+    torch.cuda.synchronize()
+    ref = O.indexed_attention(np32(x["q"][0]), np32(x["k"][0]), np32(x["v"][0]), np.arange(w.T)[None], w.scale)
+    assert_out_close(out[0], ref)
