@@ -791,8 +791,8 @@ def run_resident(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    for i in range(max(3, args.warmup)):
-        step(i % QUERY_SETS)
+    for _ in range(max(3, args.warmup)):
+        step()
     torch.cuda.synchronize()
     status = lsa.lsa_read_device_status(ws)
 
@@ -965,8 +965,8 @@ def run_prefill(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    for i in range(max(3, args.warmup)):
-        step(i % QUERY_SETS)
+    for _ in range(max(3, args.warmup)):
+        step()
     torch.cuda.synchronize()
     status = lsa.lsa_read_device_status(ws)
     e0 = torch.cuda.Event(enable_timing=True)
