@@ -11,6 +11,11 @@ torch.cuda.synchronize() on both sides; max over ranks. Inputs (2.5 GiB per
 GPU) exceed the 126 MB L2 and every step streams the 512 MiB projected-key
 cache, so no separate L2 flush is needed.
 
+On one GPU the default line also measures, in the same run, every other
+workload (the FP8 and paged steps, the L2-resident llama8b_32k and hier_1m
+steps, the 128K prefill, the scoring preparation and the two comparisons) and
+reports each one's figures under "secondary"; --no-secondary skips them.
+
 Multi-GPU: the decode step shards by sequence and KV head with no exchange, so
 each rank runs its own full workload (weak scaling, no data-path collective);
 `value` is the steps of all ranks divided by the slowest rank's time.
@@ -365,6 +370,29 @@ def run_reference(args, rank, world):
     return 0
 
 
+_SINK = None        # a list while lines are collected for the headline's "secondary" object
+_DECODE_INPUTS = {}
+
+
+def emit(line):
+    """Print one JSON line, or collect it while secondary workloads run."""
+    if _SINK is not None:
+        _SINK.append(line)
+    else:
+        print(json.dumps(line), flush=True)
+
+
+def decode_inputs(w, seed):
+    """Seeded decode inputs (host tensors, read only), generated once per
+    (workload, seed) in this process."""
+    from indexed_sparse_attention_kv_b200 import inputs as I
+
+    key = (w.name, seed)
+    if key not in _DECODE_INPUTS:
+        _DECODE_INPUTS[key] = I.make_decode_inputs(w, seed=seed)
+    return _DECODE_INPUTS[key]
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -379,7 +407,7 @@ def run_ours(args, rank, world, local_rank):
     fp8 = args.workload == "decode_128k_fp8"
     paged = args.workload == "decode_128k_paged"
     w = I.workload(WORKLOAD)
-    x = I.make_decode_inputs(w, seed=rank_seed(w, rank))
+    x = decode_inputs(w, rank_seed(w, rank))
     d = {k: x[k].to(dev) for k in ("q", "qt", "k", "v", "kt")}
     if fp8:   # the same integer values, stored as E4M3 (exact)
         d["kt8"] = d["kt"].to(torch.float8_e4m3fn)
@@ -575,7 +603,7 @@ def run_ours(args, rank, world, local_rank):
             "clocks": clocks,
             "device_status": status,
         }
-        print(json.dumps(line), flush=True)
+        emit(line)
     return 0
 
 
@@ -603,7 +631,7 @@ def run_compare(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     lsa.lib()
     w = I.workload(WORKLOAD)
-    x = I.make_decode_inputs(w, seed=rank_seed(w, rank))
+    x = decode_inputs(w, rank_seed(w, rank))
     d = {k: x[k].to(dev) for k in ("q", "qt", "k", "v", "kt")}
     qs = I.make_query_sets(w, QUERY_SETS, seed=rank_seed(w, rank) + 100)
     dq, dqt = qs["q"].to(dev), qs["qt"].to(dev)
@@ -701,7 +729,7 @@ def run_compare(args, rank, world, local_rank):
             "gpu_launches": (1 if full else 5) * steps,
             "clocks": clocks,
         }
-        print(json.dumps(line), flush=True)
+        emit(line)
     return 0
 
 
@@ -773,7 +801,7 @@ def run_resident(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     lsa.lib()
     w = I.workload(args.workload)
-    x = I.make_decode_inputs(w, seed=rank_seed(w, rank))
+    x = decode_inputs(w, rank_seed(w, rank))
     d = {k: x[k].to(dev) for k in ("q", "qt", "k", "v", "kt")}
     dims = _lib.decode_dims(d["q"], d["qt"], d["k"])
     cen = lsa.lsa_block_centroids(d["kt"], w.blk) if w.blk else None   # maintained offline, outside the step
@@ -877,7 +905,7 @@ def run_resident(args, rank, world, local_rank):
             "clocks": clocks,
             "device_status": status,
         }
-        print(json.dumps(line), flush=True)
+        emit(line)
     return 0
 
 
@@ -1036,7 +1064,7 @@ def run_prefill(args, rank, world, local_rank):
             "clocks": clocks,
             "device_status": status,
         }
-        print(json.dumps(line), flush=True)
+        emit(line)
     return 0
 
 
@@ -1192,7 +1220,7 @@ def run_prepare(args, rank, world, local_rank):
             "clocks": clocks,
             "device_status": st,
         }
-        print(json.dumps(line), flush=True)
+        emit(line)
     return 0
 
 
@@ -1261,6 +1289,73 @@ def run_ncu_case(args):
     return 0
 
 
+def run_workload(args, rank, world, local_rank):
+    if args.workload == "prefill_128k":
+        return run_prefill(args, rank, world, local_rank)
+    if args.workload == "prepare_128k":
+        return run_prepare(args, rank, world, local_rank)
+    if args.workload in RESIDENT_METRICS:
+        return run_resident(args, rank, world, local_rank)
+    if args.workload in COMPARE_METRICS:
+        return run_compare(args, rank, world, local_rank)
+    return run_ours(args, rank, world, local_rank)
+
+
+SECONDARY = ("decode_128k_fp8", "decode_128k_paged", "llama8b_32k", "hier_1m", "prefill_128k", "prepare_128k",
+             "full_kv_128k", "gather_attend_128k")
+
+
+def secondary_summary(line):
+    """The figures of one workload's line kept under the headline's
+    "secondary" object."""
+    keep = ("metric", "value", "unit", "steps", "ms_per_step", "higher_is_better", "components_ms",
+            "gather_free_sparse_step_ms", "sparse_speedup", "device_status", "gpu_launches")
+    out = {k: line[k] for k in keep if k in line}
+    out["workload"] = line.get("config", {}).get("workload")
+    roof = line.get("roofline") or {}
+    out["roofline"] = {k: roof.get(k) for k in ("bound", "kernel", "achieved", "peak", "unit", "frac")}
+    if line.get("step_roofline"):
+        out["step_roofline_frac"] = line["step_roofline"].get("frac")
+    e2e = line.get("e2e")
+    out["e2e"] = None if e2e is None else {"value": e2e.get("value"), "unit": e2e.get("unit")}
+    clk = line.get("clocks") or {}
+    out["clocks"] = {"sm_mhz": clk.get("sm_mhz"), "reasons": clk.get("reasons")}
+    return out
+
+
+def run_with_secondaries(args, rank, world, local_rank):
+    """The headline decode_128k line, then every other workload measured in
+    the same process (each with its own warm-up, CUDA-event timing and clock
+    samples; no CPU baseline), summarised under the headline's "secondary"
+    object so that one run records them all."""
+    global _SINK
+    import gc
+
+    import torch
+
+    _SINK = []
+    try:
+        rc = run_ours(args, rank, world, local_rank)
+        head = _SINK.pop() if _SINK else None
+        secondary = {}
+        for name in SECONDARY:
+            sub = argparse.Namespace(**{**vars(args), "workload": name, "no_cpu_baseline": True})
+            try:
+                run_workload(sub, rank, world, local_rank)
+                secondary[name] = secondary_summary(_SINK.pop()) if _SINK else {"error": "no line"}
+            except Exception as e:   # one failing workload must not hide the others
+                secondary[name] = {"error": f"{type(e).__name__}: {e}"[:300]}
+            gc.collect()
+            torch.cuda.empty_cache()
+    finally:
+        _SINK = None
+    _DECODE_INPUTS.clear()
+    if head is not None:
+        head["secondary"] = secondary
+        emit(head)
+    return rc
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1269,6 +1364,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="the default decode_128k line on one GPU also measures every other workload in the same "
+                         "run and reports them under \"secondary\"; this skips them")
     ap.add_argument("--workload", choices=["decode_128k", "decode_128k_fp8", "decode_128k_paged", "prefill_128k",
                                            "llama8b_32k", "hier_1m", "prepare_128k", "full_kv_128k",
                                            "gather_attend_128k"],
@@ -1302,15 +1400,9 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        if args.workload == "prefill_128k":
-            return run_prefill(args, rank, world, local_rank)
-        if args.workload == "prepare_128k":
-            return run_prepare(args, rank, world, local_rank)
-        if args.workload in RESIDENT_METRICS:
-            return run_resident(args, rank, world, local_rank)
-        if args.workload in COMPARE_METRICS:
-            return run_compare(args, rank, world, local_rank)
-        return run_ours(args, rank, world, local_rank)
+        if args.workload == "decode_128k" and world == 1 and not args.no_secondary:
+            return run_with_secondaries(args, rank, world, local_rank)
+        return run_workload(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -28,3 +28,27 @@ def test_prefill_flop():
 
 def test_prepare_bytes():
     assert bench.prepare_bytes(bench.PREPARE_SHAPE) == 1_073_741_824 + 536_870_912 + 131_072
+
+
+def test_secondary_summary_keeps_the_figures():
+    line = {"metric": "m", "value": 2.0, "unit": "steps/s", "steps": 8, "ms_per_step": 0.5, "higher_is_better": True,
+            "config": {"workload": "hier_1m", "T": 1 << 20},
+            "roofline": {"bound": "hbm", "kernel": "k", "achieved": 1.0, "peak": 2.0, "unit": "GB/s", "frac": 0.5,
+                         "traffic": None},
+            "e2e": {"value": 1.5, "unit": "steps/s", "h2d_bytes_per_step": 4},
+            "clocks": {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}, "device_status": 0}
+    s = bench.secondary_summary(line)
+    assert s["workload"] == "hier_1m" and s["value"] == 2.0 and s["ms_per_step"] == 0.5
+    assert s["roofline"]["frac"] == 0.5 and s["e2e"] == {"value": 1.5, "unit": "steps/s"}
+    assert s["clocks"]["sm_mhz"] == 1965 and s["device_status"] == 0
+
+
+def test_emit_collects_while_a_sink_is_set(capsys):
+    bench._SINK = []
+    try:
+        bench.emit({"a": 1})
+        assert bench._SINK == [{"a": 1}]
+    finally:
+        bench._SINK = None
+    bench.emit({"b": 2})
+    assert capsys.readouterr().out.strip() == '{"b": 2}'
