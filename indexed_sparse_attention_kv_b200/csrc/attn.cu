@@ -27,6 +27,14 @@
 // contained in one CTA is written directly; otherwise the CTA writes a partial
 // and the last one to finish a unit (a release/acquire counter, left at zero)
 // merges the unit's partials.
+//
+// Cluster mode (few units, as in batched decode): when every unit can own a
+// cluster of kCluster CTAs in one wave and has kCluster to 8 * kCluster tiles, CTA r
+// of unit u's cluster takes tiles r * n / kCluster .. (r + 1) * n / kCluster - 1
+// of the unit, and the cluster merges its partials through distributed shared
+// memory (each CTA produces 1 / kCluster of the unit's outputs), with no global
+// partials, counters or second pass over L2.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include "lsa_common.cuh"
@@ -36,6 +44,9 @@ namespace lsa {
 
 namespace {
 
+namespace cg = cooperative_groups;
+
+constexpr int kCluster = 8;           // CTAs per unit in cluster mode (portable size)
 constexpr int kAttnThreads = 128;
 constexpr int kAttnWarps = 4;
 constexpr int kNT = 64;               // index-set entries per tile (16 per warp)
@@ -119,7 +130,7 @@ struct AttnLayout {
     static constexpr int kTotal = kStages * kStage + kFixed;
 };
 
-template <int D, int G, bool PAGED>
+template <int D, int G, bool PAGED, int CL>
 __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
     using Lay = AttnLayout<D, G>;
     constexpr int S = Lay::kStages;
@@ -134,8 +145,12 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;    // mma fragment coordinates
     const int p = blockIdx.x;
-    const long long w0 = (long long)p * a.total_tiles / a.ctas;
-    const long long w1 = (long long)(p + 1) * a.total_tiles / a.ctas;
+    // stream-K: contiguous ranges of the flattened tiles; cluster mode: CTA r
+    // of cluster u takes its share of unit u's tiles (at least one)
+    const long long w0 = CL ? (long long)(p / CL) * a.tiles_per_unit + (long long)(p % CL) * a.tiles_per_unit / CL
+                            : (long long)p * a.total_tiles / a.ctas;
+    const long long w1 = CL ? (long long)(p / CL) * a.tiles_per_unit + (long long)(p % CL + 1) * a.tiles_per_unit / CL
+                            : (long long)(p + 1) * a.total_tiles / a.ctas;
     const int ntiles = (int)(w1 - w0);
     const size_t tstride = (size_t)a.hkv * Lay::kRowBytes;
 
@@ -345,8 +360,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
         __syncthreads();
         const int b = u / a.hkv, h = u - b * a.hkv;
         const long long wu0 = (long long)u * a.tiles_per_unit;
-        const int pfirst = owner(wu0, a);
-        const int nslot = owner(wu0 + a.tiles_per_unit - 1, a) - pfirst + 1;
+        const int pfirst = CL ? 0 : owner(wu0, a);
+        const int nslot = CL ? CL : owner(wu0 + a.tiles_per_unit - 1, a) - pfirst + 1;
         if (warp == 0) {
             float M0 = m0, M1 = m1;
 #pragma unroll
@@ -386,7 +401,28 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
                     }
                 }
             }
-            if (nslot == 1) {
+            if constexpr (CL > 0) {
+                // this CTA's partial for the cluster: the stage ring is idle (the
+                // unit's last tile is consumed and nothing is in flight)
+                float* cp = reinterpret_cast<float*>(smem);
+                if (t4 == 0) {
+                    if (g < G) {
+                        cp[g] = M0;
+                        cp[16 + g] = L0;
+                    }
+                    if (g + 8 < G) {
+                        cp[g + 8] = M1;
+                        cp[16 + g + 8] = L1;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < NTO; ++j) {
+                    const int d0 = j * 8 + 2 * t4;
+                    if (g < G) *reinterpret_cast<float2*>(cp + 32 + g * D + d0) = make_float2(acc[j][0], acc[j][1]);
+                    if (g + 8 < G)
+                        *reinterpret_cast<float2*>(cp + 32 + (g + 8) * D + d0) = make_float2(acc[j][2], acc[j][3]);
+                }
+            } else if (nslot == 1) {
                 // the whole unit lies in this CTA: write the output directly
                 const float i0 = L0 > 0.f ? 1.f / L0 : 0.f, i1 = L1 > 0.f ? 1.f / L1 : 0.f;
 #pragma unroll
@@ -421,7 +457,40 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
                 }
             }
         }
-        if (nslot > 1) {
+        if constexpr (CL > 0) {
+            // every CTA of the cluster reaches this point once (its last tile
+            // ends its only segment); merge slice r of the unit's G x D outputs
+            // from the CL partials in the cluster's shared memory
+            cg::cluster_group cluster = cg::this_cluster();
+            cluster.sync();
+            const float* parts[CL];
+#pragma unroll
+            for (int c = 0; c < CL; ++c) parts[c] = cluster.map_shared_rank(reinterpret_cast<const float*>(smem), c);
+            const int r = (int)cluster.block_rank();
+            const int e0 = r * (G * D) / CL, e1 = (r + 1) * (G * D) / CL;
+            for (int e = e0 + tid; e < e1; e += kAttnThreads) {
+                const int hd = e / D;
+                float mc[CL];
+                float M = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < CL; ++c) {
+                    mc[c] = parts[c][hd];
+                    M = fmaxf(M, mc[c]);
+                }
+                float L = 0.f, O = 0.f;
+                if (M != -INFINITY) {
+#pragma unroll
+                    for (int c = 0; c < CL; ++c) {
+                        const float wc = exp2f(mc[c] - M);
+                        L = fmaf(wc, parts[c][16 + hd], L);
+                        O = fmaf(wc, parts[c][32 + e], O);
+                    }
+                }
+                const float inv = L > 0.f ? 1.f / L : 0.f;
+                a.out[((size_t)b * a.hq + h * G) * D + e] = f2bf(O * inv);
+            }
+            cluster.sync();   // keep this CTA's partial alive for remote readers
+        } else if (nslot > 1) {
             __syncthreads();
             if (tid == 0) {
                 unsigned old;
@@ -491,19 +560,47 @@ template <int D, int G>
 cudaError_t launch_attn_t(const LaunchCtx& ctx, AttnArgs a) {
     using Lay = AttnLayout<D, G>;
     const size_t smem = Lay::kTotal;
-    auto kern = a.slots ? attn_kernel<D, G, true> : attn_kernel<D, G, false>;
-    cudaError_t e = ensure_dyn_smem((const void*)kern, (int)smem);
-    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)a.ctas);
     cfg.blockDim = dim3(kAttnThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = ctx.stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    // cluster mode when every unit has kCluster .. 8 * kCluster tiles (a few
+    // per CTA: the latency-bound regime; with more, stream-K's fuller grid
+    // streams faster) and all units' clusters are resident at once
+    if (a.tiles_per_unit >= kCluster && a.tiles_per_unit <= 8 * kCluster &&
+        (long long)a.units * kCluster <= 4ll * ctx.num_sms) {
+        auto kern = a.slots ? attn_kernel<D, G, true, kCluster> : attn_kernel<D, G, false, kCluster>;
+        cudaError_t e = ensure_dyn_smem((const void*)kern, (int)smem);
+        if (e != cudaSuccess) return e;
+        cfg.gridDim = dim3((unsigned)(a.units * kCluster));
+        // without programmatic dependent launch: clusters placed while the
+        // previous kernel's CTAs drain land on fragmented GPCs (128K decode
+        // attention 15.0 us with PDL, 14.0 us without, measured)
+        attr[0].val.programmaticStreamSerializationAllowed = 0;
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = kCluster;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+        int clusters = 0;
+        e = cached_active_clusters((const void*)kern, cfg, &clusters);
+        if (e != cudaSuccess) return e;
+        if (clusters >= a.units) {
+            e = cudaLaunchKernelEx(&cfg, kern, a);
+            if (e != cudaSuccess) return e;
+            return cudaGetLastError();
+        }
+        cfg.numAttrs = 1;
+    }
+    auto kern = a.slots ? attn_kernel<D, G, true, 0> : attn_kernel<D, G, false, 0>;
+    cudaError_t e = ensure_dyn_smem((const void*)kern, (int)smem);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3((unsigned)a.ctas);
     e = cudaLaunchKernelEx(&cfg, kern, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -48,6 +48,27 @@ inline cudaError_t cached_occupancy(const void* kern, int threads, size_t smem, 
     return e;
 }
 
+// Clusters of cfg's shape that can be resident at once (cached per kernel,
+// device and configuration).
+inline cudaError_t cached_active_clusters(const void* kern, const cudaLaunchConfig_t& cfg, int* clusters) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void*, int, unsigned, unsigned, size_t>, int> done;
+    const int dev = current_device();
+    unsigned cx = 1;
+    for (unsigned i = 0; i < cfg.numAttrs; ++i)
+        if (cfg.attrs[i].id == cudaLaunchAttributeClusterDimension) cx = cfg.attrs[i].val.clusterDim.x;
+    std::lock_guard<std::mutex> g(mu);
+    auto key = std::make_tuple(kern, dev, cfg.blockDim.x, cx, cfg.dynamicSmemBytes);
+    auto it = done.find(key);
+    if (it != done.end()) {
+        *clusters = it->second;
+        return cudaSuccess;
+    }
+    cudaError_t e = cudaOccupancyMaxActiveClusters(clusters, kern, &cfg);
+    if (e == cudaSuccess) done[key] = *clusters;
+    return e;
+}
+
 // 2-D bf16 tensor map over `outer` rows of `inner` elements, rows `row_bytes`
 // apart, boxes of box_inner x box_outer, swizzled to the box row width (32,
 // 64 or 128 bytes). Returns false if the driver entry point or the encoding
@@ -90,9 +111,11 @@ cudaError_t launch_centroids(const LaunchCtx& ctx, const uint16_t* kt, int blk, 
                              int T);
 
 // ghist (optional): the rows' histograms of key >> 21 from launch_score; the
-// kernel zeroes them after use.
+// kernel zeroes them after use. status (optional): device status word for a
+// bounded wait that ran out.
 cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int n, int B, int32_t* idx,
-                        const int32_t* blkmap, int blk, int keep, uint32_t* ghist = nullptr);
+                        const int32_t* blkmap, int blk, int keep, uint32_t* ghist = nullptr,
+                        unsigned* status = nullptr);
 
 // Scoring preparation (project.cu). y[b, t, i, :] = P[i / (H / nbases)] x[b, t, i, :]
 // for t in [t0, t0 + n) of every sequence: x [batch, T, H, d] bf16, P
