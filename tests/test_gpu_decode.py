@@ -97,7 +97,7 @@ def _topk_rows(rng, n, kind):
     raise ValueError(kind)
 
 
-@pytest.mark.parametrize("n", [1, 31, 1000, 4097, 65537, 131077, 200003])
+@pytest.mark.parametrize("n", [1, 31, 1000, 4097, 40000, 65537, 131072, 131077, 200003])
 @pytest.mark.parametrize("kind", ["ties", "nan", "signed_zero", "float", "equal", "allnan"])
 def test_topk_rows(n, kind):
     rng = np.random.default_rng(n * 7 + len(kind))
@@ -255,3 +255,65 @@ def test_attention_over_a_whole_cache():
     torch.cuda.synchronize()
     ref = O.indexed_attention(np32(x["q"][0]), np32(x["k"][0]), np32(x["v"][0]), np.arange(w.T)[None], w.scale)
     assert_out_close(out[0], ref)
+
+
+# Shapes whose attention runs in cluster mode (every unit has 8 .. 64 tiles of
+# 64 entries and all units' 8-CTA clusters fit in one wave): ragged last tiles,
+# every head dimension and group size, empty rows (NaN keys), and the paged
+# cache; the whole step is compared with the oracle.
+CLUSTER = [
+    # batch, hq, hkv, d, r, T, B
+    (1, 4, 1, 128, 64, 6000, 1000),
+    (2, 16, 2, 64, 32, 5000, 600),
+    (1, 16, 1, 256, 128, 5000, 4096),
+    (3, 6, 6, 128, 64, 3000, 513),
+    (1, 4, 2, 128, 64, 2000, 1100),
+    (2, 32, 8, 128, 64, 9000, 2048),
+]
+
+
+@pytest.mark.parametrize("case", CLUSTER, ids=[str(c) for c in CLUSTER])
+def test_decode_step_cluster_mode(case):
+    w, x = _small(case, heavy=0.05)
+    dx = to_dev(x)
+    idx, out = lsa.lsa_decode_step(dx["q"], dx["qt"], dx["k"], dx["v"], dx["kt"], w.B)
+    torch.cuda.synchronize()
+    ref_idx, ref_out = oracle_decode(x, w)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    assert_out_close(out, ref_out)
+
+
+def test_cluster_mode_empty_rows_bad_index_and_paged():
+    """Cluster mode: a head whose set is all -1 gives zeros, out-of-range
+    entries are skipped and flagged, and the paged cache gives the same bits
+    as the contiguous one."""
+    w, x = _small((2, 8, 2, 128, 64, 3000, 700), seed=11)
+    dx = to_dev(x)
+    g = torch.Generator().manual_seed(12)
+    idx = torch.stack([torch.stack([torch.randperm(w.T, generator=g)[: w.B].sort().values for _ in range(w.hkv)])
+                       for _ in range(w.batch)]).to(torch.int32)
+    idx[1, 0, :] = -1                 # an empty set
+    idx[0, 1, 5] = w.T                # out of range: skipped, flagged
+    ws = lsa.workspace(lsa._lib.decode_dims(dx["q"], dx["qt"], dx["k"]), w.B)
+    out = lsa.lsa_indexed_attn(dx["q"], dx["k"], dx["v"], idx.cuda(), ws=ws)
+    torch.cuda.synchronize()
+    assert lsa.lsa_read_device_status(ws) & lsa._lib.DEV_BAD_INDEX
+    ref_idx = idx.numpy().copy()
+    ref_idx[ref_idx >= w.T] = -1
+    for b in range(w.batch):
+        ref = O.indexed_attention(np32(x["q"][b]), np32(x["k"][b]), np32(x["v"][b]), ref_idx[b], w.scale)
+        assert_out_close(out[b], ref)
+    assert torch.all(out[1, :4] == 0)
+    # paged: the same rows in a shuffled pool
+    n = w.batch * w.T
+    perm = torch.randperm(n, generator=torch.Generator().manual_seed(13)).cuda()
+    kp = torch.empty((n, w.hkv, w.d), dtype=torch.bfloat16, device="cuda")
+    vp = torch.empty_like(kp)
+    kp[perm] = dx["k"].reshape(n, w.hkv, w.d)
+    vp[perm] = dx["v"].reshape(n, w.hkv, w.d)
+    idx_ok = idx.clone()
+    idx_ok[idx_ok >= w.T] = -1
+    out_c = lsa.lsa_indexed_attn(dx["q"], dx["k"], dx["v"], idx_ok.cuda())
+    out_p = lsa.lsa_indexed_attn_paged(dx["q"], kp, vp, perm.to(torch.int32).view(w.batch, w.T), idx_ok.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(out_c, out_p)
