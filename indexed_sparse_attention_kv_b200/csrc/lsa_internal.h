@@ -111,11 +111,9 @@ cudaError_t launch_centroids(const LaunchCtx& ctx, const uint16_t* kt, int blk, 
                              int T);
 
 // ghist (optional): the rows' histograms of key >> 21 from launch_score; the
-// kernel zeroes them after use. status (optional): device status word for a
-// bounded wait that ran out.
+// kernel zeroes them after use.
 cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int n, int B, int32_t* idx,
-                        const int32_t* blkmap, int blk, int keep, uint32_t* ghist = nullptr,
-                        unsigned* status = nullptr);
+                        const int32_t* blkmap, int blk, int keep, uint32_t* ghist = nullptr);
 
 // Scoring preparation (project.cu). y[b, t, i, :] = P[i / (H / nbases)] x[b, t, i, :]
 // for t in [t0, t0 + n) of every sequence: x [batch, T, H, d] bf16, P
