@@ -77,3 +77,31 @@ def test_fp8_decode_128k_full_size():
     torch.cuda.synchronize()
     assert torch.equal(idx8, idx16)
     assert torch.equal(out8, out16)
+
+
+def test_fp8_nan_keys_are_never_selected():
+    """E4M3 NaN keys (in any channel) give NaN scores, as in the bf16 path, and
+    are never selected; every other score is identical."""
+    w, x = _case((2, 32, 8, 128, 64, 3000, 400), seed=33)
+    g = torch.Generator().manual_seed(34)
+    n_nan = 300
+    b = torch.randint(0, w.batch, (n_nan,), generator=g)
+    t = torch.randint(0, w.T, (n_nan,), generator=g)
+    h = torch.randint(0, w.hkv, (n_nan,), generator=g)
+    c = torch.randint(0, w.r, (n_nan,), generator=g)
+    x["kt"][b, t, h, c] = float("nan")
+    d = to_dev(x)
+    kt8 = x["kt"].to(torch.float8_e4m3fn).cuda()
+    s16 = lsa.lsa_score(d["qt"], d["kt"])
+    s8 = lsa.lsa_score_fp8(d["qt"], kt8)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.isnan(s8), torch.isnan(s16))
+    assert int(torch.isnan(s8).sum()) > 0
+    ok = ~torch.isnan(s16)
+    assert torch.equal(s8[ok], s16[ok])
+    idx8, out8 = lsa.lsa_decode_step_fp8(d["q"], d["qt"], d["k"], d["v"], kt8, w.B)
+    idx16, out16 = lsa.lsa_decode_step(d["q"], d["qt"], d["k"], d["v"], d["kt"], w.B)
+    torch.cuda.synchronize()
+    assert torch.equal(idx8, idx16) and torch.equal(out8, out16)
+    ref_idx, ref_out = oracle_decode(x, w)
+    assert np.array_equal(idx8.cpu().numpy(), ref_idx)
