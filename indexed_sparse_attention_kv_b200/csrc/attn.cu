@@ -29,11 +29,11 @@
 // merges the unit's partials.
 //
 // Cluster mode (few units, as in batched decode): when every unit can own a
-// cluster of kCluster CTAs in one wave and has kCluster to 8 * kCluster tiles, CTA r
-// of unit u's cluster takes tiles r * n / kCluster .. (r + 1) * n / kCluster - 1
-// of the unit, and the cluster merges its partials through distributed shared
-// memory (each CTA produces 1 / kCluster of the unit's outputs), with no global
-// partials, counters or second pass over L2.
+// cluster of C CTAs (16, else 8) in one wave and has C to 8 * C tiles, CTA r of
+// unit u's cluster takes tiles r * n / C .. (r + 1) * n / C - 1 of the unit,
+// and the cluster merges its partials through distributed shared memory (each
+// CTA produces 1 / C of the unit's outputs), with no global partials, counters
+// or second pass over L2.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
@@ -46,7 +46,6 @@ namespace {
 
 namespace cg = cooperative_groups;
 
-constexpr int kCluster = 8;           // CTAs per unit in cluster mode (portable size)
 constexpr int kAttnThreads = 128;
 constexpr int kAttnWarps = 4;
 constexpr int kNT = 64;               // index-set entries per tile (16 per warp)
@@ -556,51 +555,78 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
     cp_async_wait<0>();
 }
 
-template <int D, int G>
-cudaError_t launch_attn_t(const LaunchCtx& ctx, AttnArgs a) {
-    using Lay = AttnLayout<D, G>;
-    const size_t smem = Lay::kTotal;
+// Launches cluster mode with CL-CTA clusters if every unit has CL .. 8 * CL
+// tiles (a few per CTA: the latency-bound regime; with more, stream-K's fuller
+// grid streams faster) and all units' clusters are resident at once; *done
+// tells whether it launched.
+template <int D, int G, int CL>
+cudaError_t try_cluster(const LaunchCtx& ctx, const AttnArgs& a, bool* done) {
+    *done = false;
+    if (a.tiles_per_unit < CL || a.tiles_per_unit > 8 * CL || (long long)a.units * CL > 4ll * ctx.num_sms)
+        return cudaSuccess;
+    const size_t smem = AttnLayout<D, G>::kTotal;
+    auto kern = a.slots ? attn_kernel<D, G, true, CL> : attn_kernel<D, G, false, CL>;
+    cudaError_t e = ensure_dyn_smem((const void*)kern, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (CL > 8) {   // beyond the portable cluster size
+        static std::mutex mu;
+        static std::map<std::pair<const void*, int>, bool> allowed;
+        std::lock_guard<std::mutex> g(mu);
+        bool& ok = allowed[{(const void*)kern, current_device()}];
+        if (!ok) {
+            e = cudaFuncSetAttribute((const void*)kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+            ok = true;
+        }
+    }
     cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(a.units * CL));
     cfg.blockDim = dim3(kAttnThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = ctx.stream;
-    cudaLaunchAttribute attr[2];
+    // without programmatic dependent launch: clusters placed while the
+    // previous kernel's CTAs drain land on fragmented GPCs (128K decode
+    // attention 15.0 us with PDL, 14.0 us without, measured)
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    e = cached_active_clusters((const void*)kern, cfg, &clusters);
+    if (e != cudaSuccess) return e;
+    if (clusters < a.units) return cudaSuccess;
+    e = cudaLaunchKernelEx(&cfg, kern, a);
+    if (e != cudaSuccess) return e;
+    *done = true;
+    return cudaGetLastError();
+}
+
+template <int D, int G>
+cudaError_t launch_attn_t(const LaunchCtx& ctx, AttnArgs a) {
+    // cluster mode: 16-CTA clusters (two tiles or more per CTA) when they all
+    // fit, else 8-CTA clusters; otherwise stream-K
+    bool done = false;
+    cudaError_t e = try_cluster<D, G, 16>(ctx, a, &done);
+    if (e != cudaSuccess || done) return e;
+    e = try_cluster<D, G, 8>(ctx, a, &done);
+    if (e != cudaSuccess || done) return e;
+    const size_t smem = AttnLayout<D, G>::kTotal;
+    auto kern = a.slots ? attn_kernel<D, G, true, 0> : attn_kernel<D, G, false, 0>;
+    e = ensure_dyn_smem((const void*)kern, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)a.ctas);
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = ctx.stream;
+    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // cluster mode when every unit has kCluster .. 8 * kCluster tiles (a few
-    // per CTA: the latency-bound regime; with more, stream-K's fuller grid
-    // streams faster) and all units' clusters are resident at once
-    if (a.tiles_per_unit >= kCluster && a.tiles_per_unit <= 8 * kCluster &&
-        (long long)a.units * kCluster <= 4ll * ctx.num_sms) {
-        auto kern = a.slots ? attn_kernel<D, G, true, kCluster> : attn_kernel<D, G, false, kCluster>;
-        cudaError_t e = ensure_dyn_smem((const void*)kern, (int)smem);
-        if (e != cudaSuccess) return e;
-        cfg.gridDim = dim3((unsigned)(a.units * kCluster));
-        // without programmatic dependent launch: clusters placed while the
-        // previous kernel's CTAs drain land on fragmented GPCs (128K decode
-        // attention 15.0 us with PDL, 14.0 us without, measured)
-        attr[0].val.programmaticStreamSerializationAllowed = 0;
-        attr[1].id = cudaLaunchAttributeClusterDimension;
-        attr[1].val.clusterDim.x = kCluster;
-        attr[1].val.clusterDim.y = 1;
-        attr[1].val.clusterDim.z = 1;
-        cfg.numAttrs = 2;
-        int clusters = 0;
-        e = cached_active_clusters((const void*)kern, cfg, &clusters);
-        if (e != cudaSuccess) return e;
-        if (clusters >= a.units) {
-            e = cudaLaunchKernelEx(&cfg, kern, a);
-            if (e != cudaSuccess) return e;
-            return cudaGetLastError();
-        }
-        cfg.numAttrs = 1;
-    }
-    auto kern = a.slots ? attn_kernel<D, G, true, 0> : attn_kernel<D, G, false, 0>;
-    cudaError_t e = ensure_dyn_smem((const void*)kern, (int)smem);
-    if (e != cudaSuccess) return e;
-    cfg.gridDim = dim3((unsigned)a.ctas);
     e = cudaLaunchKernelEx(&cfg, kern, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
