@@ -612,11 +612,14 @@ cudaError_t launch_topk(const LaunchCtx& ctx, const float* scores, int rows, int
     a.B = B;
     a.blk = blk;
     a.keep = keep;
-    // rows of up to 16K keys: one 1024-thread CTA per row (measured faster
-    // than 256 or 512 threads for 4K-key rows: the selection's passes and
-    // barriers, not the loads, set its time)
+    // rows of up to 4K keys, and up to 16K keys unless the set is short: one
+    // 1024-thread CTA per row (measured faster than 256 or 512 threads for
+    // 4K-key rows: the selection's passes and barriers, not the loads, set
+    // its time). A short set from a longer row (B <= n / 16, as the coarse
+    // stage's kept blocks) goes to the cluster instead, whose CTAs share the
+    // row while its lists stay short.
     if (n <= 1024 * 4) return launch_small<1024, 4>(ctx, a, rows);
-    if (n <= 1024 * kSmallItems) return launch_small<1024, kSmallItems>(ctx, a, rows);
+    if (n <= 1024 * kSmallItems && (long long)B * 16 > n) return launch_small<1024, kSmallItems>(ctx, a, rows);
     // Cluster size: about 16K keys per CTA, at most 8 (portable); fewer CTAs
     // per row when there are many rows.
     int cs = 1;
