@@ -574,8 +574,11 @@ cudaError_t try_cluster(const LaunchCtx& ctx, const AttnArgs& a, bool* done) {
         std::lock_guard<std::mutex> g(mu);
         bool& ok = allowed[{(const void*)kern, current_device()}];
         if (!ok) {
-            e = cudaFuncSetAttribute((const void*)kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-            if (e != cudaSuccess) return e;
+            if (cudaFuncSetAttribute((const void*)kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess) {
+                (void)cudaGetLastError();   // not offered: the caller tries the portable size
+                return cudaSuccess;
+            }
             ok = true;
         }
     }
@@ -595,8 +598,10 @@ cudaError_t try_cluster(const LaunchCtx& ctx, const AttnArgs& a, bool* done) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int clusters = 0;
-    e = cached_active_clusters((const void*)kern, cfg, &clusters);
-    if (e != cudaSuccess) return e;
+    if (cached_active_clusters((const void*)kern, cfg, &clusters) != cudaSuccess) {
+        (void)cudaGetLastError();   // no answer: the caller falls back to a smaller cluster or stream-K
+        return cudaSuccess;
+    }
     if (clusters < a.units) return cudaSuccess;
     e = cudaLaunchKernelEx(&cfg, kern, a);
     if (e != cudaSuccess) return e;
