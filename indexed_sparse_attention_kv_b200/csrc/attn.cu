@@ -29,7 +29,8 @@
 // merges the unit's partials.
 //
 // Cluster mode (few units, as in batched decode): when every unit can own a
-// cluster of C CTAs (16, else 8) in one wave and has C to 8 * C tiles, CTA r of
+// cluster of C CTAs (16, else 8) in one wave and has C to 4 * C (C = 16) or
+// 8 * C (C = 8) tiles, CTA r of
 // unit u's cluster takes tiles r * n / C .. (r + 1) * n / C - 1 of the unit,
 // and the cluster merges its partials through distributed shared memory (each
 // CTA produces 1 / C of the unit's outputs), with no global partials, counters
@@ -556,13 +557,15 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
 }
 
 // Launches cluster mode with CL-CTA clusters if every unit has CL .. 8 * CL
-// tiles (a few per CTA: the latency-bound regime; with more, stream-K's fuller
-// grid streams faster) and all units' clusters are resident at once; *done
-// tells whether it launched.
+// tiles (CL .. 4 * CL for 16-CTA clusters: a few per CTA, the latency-bound
+// regime; with more, stream-K's fuller grid streams as fast or faster,
+// measured over batch 1-8 and B 512-8192 at 128K) and all units' clusters are
+// resident at once; *done tells whether it launched.
 template <int D, int G, int CL>
 cudaError_t try_cluster(const LaunchCtx& ctx, const AttnArgs& a, bool* done) {
     *done = false;
-    if (a.tiles_per_unit < CL || a.tiles_per_unit > 8 * CL || (long long)a.units * CL > 4ll * ctx.num_sms)
+    const int max_per_cta = CL > 8 ? 4 : 8;
+    if (a.tiles_per_unit < CL || a.tiles_per_unit > max_per_cta * CL || (long long)a.units * CL > 4ll * ctx.num_sms)
         return cudaSuccess;
     const size_t smem = AttnLayout<D, G>::kTotal;
     auto kern = a.slots ? attn_kernel<D, G, true, CL> : attn_kernel<D, G, false, CL>;
