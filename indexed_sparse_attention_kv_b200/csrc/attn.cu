@@ -30,11 +30,10 @@
 //
 // Cluster mode (few units, as in batched decode): when every unit can own a
 // cluster of C CTAs (16, else 8) in one wave and has C to 4 * C (C = 16) or
-// 8 * C (C = 8) tiles, CTA r of
-// unit u's cluster takes tiles r * n / C .. (r + 1) * n / C - 1 of the unit,
-// and the cluster merges its partials through distributed shared memory (each
-// CTA produces 1 / C of the unit's outputs), with no global partials, counters
-// or second pass over L2.
+// 8 * C (C = 8) tiles, CTA r of unit u's cluster takes tiles r * n / C ..
+// (r + 1) * n / C - 1 of the unit, and the cluster merges its partials through
+// distributed shared memory (each CTA produces 1 / C of the unit's outputs),
+// with no global partials, counters or second pass over L2.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
