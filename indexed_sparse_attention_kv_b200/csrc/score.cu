@@ -50,20 +50,22 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two) {
     return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
-// 16 E4M3 values . q[0..16), fp32 accumulation in channel order.
+// 16 E4M3 values . q[0..16), fp32 accumulation in two interleaved chains (even
+// and odd channels, summed at the end) so that consecutive FMAs do not wait on
+// each other.
 __device__ __forceinline__ float dot16_e4m3(const uint4 w, const float* q) {
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-    float acc = 0.f;
+    float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const float2 f0 = e4m3x2_to_float2(ws[i]);
         const float2 f1 = e4m3x2_to_float2(ws[i] >> 16);
-        acc = fmaf(q[4 * i + 0], f0.x, acc);
-        acc = fmaf(q[4 * i + 1], f0.y, acc);
-        acc = fmaf(q[4 * i + 2], f1.x, acc);
-        acc = fmaf(q[4 * i + 3], f1.y, acc);
+        acc0 = fmaf(q[4 * i + 0], f0.x, acc0);
+        acc1 = fmaf(q[4 * i + 1], f0.y, acc1);
+        acc0 = fmaf(q[4 * i + 2], f1.x, acc0);
+        acc1 = fmaf(q[4 * i + 3], f1.y, acc1);
     }
-    return acc;
+    return acc0 + acc1;
 }
 
 __device__ __forceinline__ float dot8(const uint4 w, const float* q) {
