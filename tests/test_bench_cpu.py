@@ -1,6 +1,9 @@
-"""Host-side pins of bench.py's algorithmic byte and flop counts against the
-figures the design states for each workload (closed forms of the shapes)."""
+"""Host-side checks of bench.py: its algorithmic byte and flop counts against
+the closed forms of each workload's shapes, the secondary-workload summary and
+line collection, and the reference arm's JSON line (the oracle on the host)."""
 from __future__ import annotations
+
+import json
 
 import bench
 from indexed_sparse_attention_kv_b200 import inputs as I
@@ -52,3 +55,27 @@ def test_emit_collects_while_a_sink_is_set(capsys):
         bench._SINK = None
     bench.emit({"b": 2})
     assert capsys.readouterr().out.strip() == '{"b": 2}'
+
+
+def _reference_line(capsys, *argv):
+    assert bench.main(["--impl", "reference", *argv]) == 0
+    out = capsys.readouterr().out.strip().splitlines()
+    assert len(out) == 1
+    return json.loads(out[0])
+
+
+def test_reference_arm_line(capsys):
+    """The reference arm (the oracle on the host cores) prints one line with
+    the contract's keys; steps x ms_per_step is its timed region."""
+    d = _reference_line(capsys, "--workload", "llama8b_32k", "--steps", "1", "--warmup", "1")
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1
+    assert d["unit"] == "steps/s" and d["higher_is_better"] is True
+    assert abs(d["value"] - 1e3 / d["ms_per_step"]) <= 1e-6 * d["value"]
+    assert d["config"]["workload"] == "llama8b_32k" and "parallelism" in d["config"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_comparators_unavailable(capsys):
+    d = _reference_line(capsys, "--workload", "full_kv_128k")
+    assert d["impl"] == "reference" and "unavailable" in d
