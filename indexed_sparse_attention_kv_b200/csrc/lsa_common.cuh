@@ -39,6 +39,14 @@ __device__ __forceinline__ uint32_t score_key(float x) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Order key -> the smallest float with that key (keys of NaN patterns -> -inf),
+// so that s >= key_floor(k) <=> score_key(s) >= k for every non-NaN s.
+__device__ __forceinline__ float key_floor(uint32_t k) {
+    if (k & 0x80000000u) return __uint_as_float(k & 0x7FFFFFFFu);
+    if (k <= 0x007FFFFFu) return -__int_as_float(0x7f800000);
+    return __uint_as_float(~k);
+}
+
 // ---------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -103,14 +103,6 @@ __device__ __forceinline__ Unit decode_unit(int u, const GemmArgs& a) {
     return t;
 }
 
-// Order key -> the smallest float with that key (keys of NaN patterns -> -inf),
-// so that s >= key_floor(k) <=> score_key(s) >= k for every non-NaN s.
-__device__ __forceinline__ float key_floor(uint32_t k) {
-    if (k & 0x80000000u) return __uint_as_float(k & 0x7FFFFFFFu);
-    if (k <= 0x007FFFFFu) return -__int_as_float(0x7f800000);
-    return __uint_as_float(~k);
-}
-
 // ---------------------------------------------------------------- score GEMM
 // D[128 queries, 256 keys] = Qbar_h[rows] . Kt_h[cols]^T per tile, K = r.
 // Shared memory: two A slots (one per unit, double-buffered), `stages` B

@@ -175,6 +175,33 @@ __device__ __forceinline__ void load_batch(const float* src, bool vec, int i00, 
     }
 }
 
+// As load_batch, the raw scores (NaN past `end`): the list pass compares them
+// with a float threshold and converts only its hits to order keys.
+__device__ __forceinline__ void load_batch_f(const float* src, bool vec, int i00, int end, int lane,
+                                             float (&ff)[kBatch][4]) {
+    if (vec && i00 + 128 * kBatch <= end) {
+        float4 v[kBatch];
+#pragma unroll
+        for (int ub = 0; ub < kBatch; ++ub)
+            v[ub] = __ldcg(reinterpret_cast<const float4*>(src + i00 + ub * 128 + lane * 4));
+#pragma unroll
+        for (int ub = 0; ub < kBatch; ++ub) {
+            ff[ub][0] = v[ub].x;
+            ff[ub][1] = v[ub].y;
+            ff[ub][2] = v[ub].z;
+            ff[ub][3] = v[ub].w;
+        }
+    } else {
+#pragma unroll
+        for (int ub = 0; ub < kBatch; ++ub)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i00 + ub * 128 + lane * 4 + u;
+                ff[ub][u] = i < end ? __ldcg(src + i) : __int_as_float(0x7fc00000);
+            }
+    }
+}
+
 template <bool EXT_HIST>
 __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster_kernel(const TopkArgs a) {
     cg::cluster_group cluster = cg::this_cluster();
@@ -227,25 +254,28 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster_kernel(const Top
     // ---- 2. per-warp lists of (key, position) with bin >= b0, in position order
     // Coalesced steps of 128 keys (lane: 4 consecutive keys, one 16-byte load;
     // every load of a batch issued before any use); four ballots per step give
-    // each hit its rank in position order without a shuffle scan.
+    // each hit its rank in position order without a shuffle scan. A score is
+    // in bin >= b0 iff it is >= the smallest float of bin b0 (NaN: never), so
+    // only the hits are converted to order keys.
     uint32_t* wkey = sh.lkey + warp * kListPerWarp;
     int* wpos = sh.lpos + warp * kListPerWarp;
     int wc = 0;
     const unsigned lt = (1u << lane) - 1u;
+    const float thr_b0 = key_floor(b0 << 21);
     for (int i00 = wbeg; i00 < wend; i00 += 128 * kBatch) {
-        uint32_t kk[kBatch][4];
-        load_batch(src, vec, i00, wend, lane, kk);
+        float ff[kBatch][4];
+        load_batch_f(src, vec, i00, wend, lane, ff);
 #pragma unroll
         for (int ub = 0; ub < kBatch; ++ub) {
             unsigned m[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) m[u] = __ballot_sync(0xffffffffu, kk[ub][u] != 0u && (kk[ub][u] >> 21) >= b0);
+            for (int u = 0; u < 4; ++u) m[u] = __ballot_sync(0xffffffffu, ff[ub][u] >= thr_b0);
             int slot = wc + __popc(m[0] & lt) + __popc(m[1] & lt) + __popc(m[2] & lt) + __popc(m[3] & lt);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 if ((m[u] >> lane) & 1u) {
                     if (slot < kListPerWarp) {
-                        wkey[slot] = kk[ub][u];
+                        wkey[slot] = score_key(ff[ub][u]);
                         wpos[slot] = base + i00 + ub * 128 + lane * 4 + u;
                     }
                     ++slot;
