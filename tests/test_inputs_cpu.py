@@ -51,3 +51,18 @@ def test_projection_inputs():
     assert torch.equal(a["x"], b["x"]) and torch.equal(a["P"], b["P"])
     assert a["x"].shape == (1, 10, 4, 16) and a["P"].shape == (2, 8, 16)
     assert a["x"].float().abs().max() <= 3 and a["P"].float().abs().max() <= 2
+
+
+def test_query_sets_seeded_distinct_and_in_range():
+    """Rotating query sets: deterministic per seed, set i from seed + i (so the
+    sets differ), projected queries integers in [-R, R], queries bf16."""
+    w = _small(0.0)
+    a, b = I.make_query_sets(w, 3, seed=500), I.make_query_sets(w, 3, seed=500)
+    assert torch.equal(a["q"], b["q"]) and torch.equal(a["qt"], b["qt"])
+    assert a["q"].shape == (3, 2, 8, 16) and a["qt"].shape == (3, 2, 8, 8)
+    assert not torch.equal(a["qt"][0], a["qt"][1]) and not torch.equal(a["q"][1], a["q"][2])
+    c = I.make_query_sets(w, 1, seed=501)   # set 1 of seed 500 is set 0 of seed 501
+    assert torch.equal(c["qt"][0], a["qt"][1]) and torch.equal(c["q"][0], a["q"][1])
+    v = a["qt"].float()
+    assert torch.equal(v, v.round()) and v.abs().max() <= w.int_range
+    assert a["q"].dtype == torch.bfloat16
