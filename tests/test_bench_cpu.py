@@ -79,3 +79,41 @@ def test_reference_arm_line(capsys):
 def test_reference_arm_comparators_unavailable(capsys):
     d = _reference_line(capsys, "--workload", "full_kv_128k")
     assert d["impl"] == "reference" and "unavailable" in d
+
+
+def test_secondary_workloads_are_collected_into_the_headline(capsys, monkeypatch):
+    """run_with_secondaries: the headline line is printed once, with every other
+    workload's summary under "secondary"; a workload that raises is recorded
+    as an error instead of hiding the others (host logic only: the GPU runs
+    are replaced by stubs that emit lines)."""
+    import argparse
+    import sys
+    import types
+
+    fake_torch = types.SimpleNamespace(cuda=types.SimpleNamespace(empty_cache=lambda: None))
+    monkeypatch.setitem(sys.modules, "torch", fake_torch)
+
+    def fake_ours(args, rank, world, local_rank):
+        bench.emit({"metric": "m", "value": 1.0, "unit": "steps/s", "config": {"workload": "decode_128k"}})
+        return 0
+
+    def fake_workload(args, rank, world, local_rank):
+        if args.workload == "hier_1m":
+            raise RuntimeError("boom")
+        assert args.no_cpu_baseline
+        bench.emit({"metric": args.workload, "value": 2.0, "unit": "u", "steps": 3, "ms_per_step": 0.5,
+                    "config": {"workload": args.workload}, "roofline": {"frac": 0.5}})
+        return 0
+
+    monkeypatch.setattr(bench, "run_ours", fake_ours)
+    monkeypatch.setattr(bench, "run_workload", fake_workload)
+    args = argparse.Namespace(workload="decode_128k", no_cpu_baseline=False, steps=3, warmup=3)
+    assert bench.run_with_secondaries(args, 0, 1, 0) == 0
+    lines = capsys.readouterr().out.strip().splitlines()
+    assert len(lines) == 1
+    head = json.loads(lines[0])
+    assert head["metric"] == "m" and set(head["secondary"]) == set(bench.SECONDARY)
+    assert head["secondary"]["hier_1m"] == {"error": "RuntimeError: boom"}
+    assert head["secondary"]["llama8b_32k"]["value"] == 2.0
+    assert head["secondary"]["llama8b_32k"]["workload"] == "llama8b_32k"
+    assert bench._SINK is None
